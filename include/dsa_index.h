@@ -1,0 +1,120 @@
+/*
+ * dsa_index.h - C ABI of the B200 lightning-indexer library (libdsa_index.so).
+ *
+ * The library computes, for query rows t and keys s, the DeepSeek Sparse
+ * Attention lightning-indexer score
+ *
+ *     I(t,s) = sum_{j<H} w(t,j) * ReLU(q(t,j) . k(s))
+ *
+ * ("DeepSeek DSA FLOPs", Lightning Indexer, eq. index score: H index heads of
+ * width d share one key vector per position) and returns, per query row, the
+ * exact Top-k keys among the causally visible ones.  A query at absolute
+ * position p sees keys 0..p ("DeepSeek DSA FLOPs", causal token-pair count,
+ * N_dense = T(T+1)/2) and keeps m = min(k, p+1) of them (N_sel).
+ *
+ * Conventions shared by every entry point
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    the caller owns all of them.  Inputs are read-only; outputs are fully
+ *    overwritten.  The library allocates no memory: scratch comes from the
+ *    caller's workspace, sized by the matching *_workspace_bytes() call.
+ *  - Layouts are row-major and contiguous.  q/k hold bf16 values as raw
+ *    16-bit patterns; w is fp32.  q, k and the workspace must be 16-byte
+ *    aligned (TMA), w/out_* 4-byte aligned.
+ *  - Outputs per row: out_idx[row][0..topk) int32 key indices and
+ *    out_score[row][0..topk) fp32 scores, sorted by score descending, ties by
+ *    smaller key index; entries past m are idx = -1, score = -inf.
+ *  - Scores are fp32: dot products accumulate in fp32 on the tensor cores
+ *    from the exact bf16 inputs; the head sum is the fp32 chain
+ *    acc = fmaf(w_j, max(dot_j, 0), acc) for j = 0..H-1 from acc = +0.
+ *  - Supported: d == 128, H in {32, 64}, 1 <= topk <= 2048, key counts
+ *    below 2^31.  Inputs must be finite (non-finite inputs never fault or
+ *    hang, but their order is unspecified).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) unless stated otherwise, and returns a status:
+ */
+#ifndef DSA_INDEX_H
+#define DSA_INDEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_OK 0
+#define DSA_EINVAL (-1)       /* null pointer, negative/inconsistent sizes, misalignment */
+#define DSA_EUNSUPPORTED (-2) /* d != 128, H not in {32, 64}, topk outside [1, 2048] */
+#define DSA_EWORKSPACE (-3)   /* ws_bytes below the *_workspace_bytes() requirement */
+#define DSA_ESEED (-4)        /* (pruned) bad seed list: see dsa_index_prefill_pruned */
+#define DSA_ECUDA (-5)        /* a CUDA runtime call failed: see dsa_last_error_string() */
+#define DSA_EDEVICE (-6)      /* a device-side check failed (reported by synchronous calls) */
+
+/* Counters of the pruned (DoSA) path; all are sums over the call's rows. */
+typedef struct dsa_stats {
+  int64_t screened_pairs; /* non-seed visible (row, key) pairs given an upper bound */
+  int64_t survivor_pairs; /* screened pairs whose bound reached the threshold */
+  int64_t refined_pairs;  /* survivor pairs scored exactly with all heads */
+  int64_t records;        /* records written for the final selection (seed + refined) */
+  int64_t recovered_rows; /* rows recomputed by the dense path after a capacity overflow */
+} dsa_stats;
+
+/* Text of the last error seen by this library in the calling thread. */
+DSA_API const char* dsa_last_error_string(void);
+
+/*
+ * Chunked causal prefill ("DeepSeek DSA FLOPs", Full-prefix index scoring and
+ * Prefill / training): query row t (0 <= t < T_q) sits at absolute position
+ * q_offset + t and scores keys 0..q_offset+t of k.
+ *   q          device, [T_q][H][d] bf16
+ *   w          device, [T_q][H] fp32 head weights, used as given
+ *   k          device, [T_k][d] bf16 keys; requires 0 <= q_offset,
+ *              q_offset + T_q <= T_k
+ *   out_idx    device, [T_q][topk] int32
+ *   out_score  device, [T_q][topk] fp32
+ *   workspace  device, at least dsa_index_prefill_workspace_bytes() bytes
+ * T_q == 0 is a no-op.
+ */
+DSA_API size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk);
+DSA_API int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                      int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
+                      float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Batched decode ("DeepSeek DSA FLOPs", Decode): sequence b has one new query
+ * q[b] (H rows) and its own key cache k_cache[b] of capacity t_cap, of which
+ * the first seq_len[b] keys are visible (the new token's key included).
+ *   q          device, [B][H][d] bf16
+ *   w          device, [B][H] fp32
+ *   k_cache    device, [B][t_cap][d] bf16
+ *   seq_len    device, [B] int32, 0 <= seq_len[b] <= t_cap (a length outside
+ *              that range is treated as 0 and sets the device status word)
+ *   out_idx    device, [B][topk] int32 key positions within the sequence
+ *   out_score  device, [B][topk] fp32
+ * Requires 1 <= B <= 65536 and B * t_cap < 2^31.
+ */
+DSA_API size_t dsa_index_decode_workspace_bytes(int B, int64_t t_cap, int H, int d, int topk);
+DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
+                     const int32_t* seq_len, int B, int64_t t_cap, int H, int d, int topk,
+                     int32_t* out_idx, float* out_score, void* workspace, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * Device status word of the most recent call that used `workspace`: 0 when
+ * every device-side check passed.  Synchronises `stream`.
+ * Bit 0: a bounded wait inside a kernel gave up (the kernel unwound).
+ * Bit 1: a capacity or length check failed.  Bit 2: the seed list was invalid.
+ */
+DSA_API int dsa_index_device_status(const void* workspace, uint32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEX_H */

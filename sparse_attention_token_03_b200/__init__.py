@@ -1,0 +1,177 @@
+"""B200 (sm_100a) lightning-indexer scoring with exact Top-k.
+
+Python binding of libdsa_index.so (include/dsa_index.h).  This module only
+marshals arguments: it checks dtypes, shapes, devices and contiguity of torch
+tensors, allocates outputs and the workspace through torch, and passes raw
+pointers plus the current CUDA stream to the C ABI.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
+    "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
+    "dsa_index_device_status",
+]
+
+DSA_OK = 0
+STATUS_NAMES = {
+    -1: "DSA_EINVAL", -2: "DSA_EUNSUPPORTED", -3: "DSA_EWORKSPACE", -4: "DSA_ESEED",
+    -5: "DSA_ECUDA", -6: "DSA_EDEVICE",
+}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libdsa_index.so (building it first if it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if build_if_missing and _build.stale():
+            _build.build()
+        if not path.exists():
+            raise RuntimeError(f"{path} is missing; run sparse_attention_token_03_b200/build.py")
+        L = ctypes.CDLL(str(path))
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.dsa_last_error_string.restype = ctypes.c_char_p
+        L.dsa_index_prefill_workspace_bytes.argtypes = [I64, I64, I, I, I]
+        L.dsa_index_prefill_workspace_bytes.restype = SZ
+        L.dsa_index_prefill.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_prefill.restype = I
+        L.dsa_index_decode_workspace_bytes.argtypes = [I, I64, I, I, I]
+        L.dsa_index_decode_workspace_bytes.restype = SZ
+        L.dsa_index_decode.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_decode.restype = I
+        L.dsa_index_device_status.argtypes = [P, P, P]
+        L.dsa_index_device_status.restype = I
+        _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != DSA_OK:
+        raise DSAError(rc, lib().dsa_last_error_string().decode())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if t.device.type != "cuda" or (device is not None and t.device != device):
+        raise ValueError(f"{name} must be on {device or 'a CUDA device'}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def dsa_index_prefill_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int) -> int:
+    return int(lib().dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk))
+
+
+def dsa_index_decode_workspace_bytes(B: int, t_cap: int, H: int, d: int, topk: int) -> int:
+    return int(lib().dsa_index_decode_workspace_bytes(B, t_cap, H, d, topk))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is None:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8, 1, device)
+    return workspace
+
+
+def _outputs(rows: int, topk: int, device, out_idx, out_score):
+    if out_idx is None:
+        out_idx = torch.empty((rows, topk), dtype=torch.int32, device=device)
+    if out_score is None:
+        out_score = torch.empty((rows, topk), dtype=torch.float32, device=device)
+    _need(out_idx, "out_idx", torch.int32, 2, device)
+    _need(out_score, "out_score", torch.float32, 2, device)
+    if tuple(out_idx.shape) != (rows, topk) or tuple(out_score.shape) != (rows, topk):
+        raise ValueError(f"outputs must be ({rows}, {topk})")
+    return out_idx, out_score
+
+
+def dsa_index_prefill(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offset: int, topk: int,
+                      out_idx=None, out_score=None, workspace=None):
+    """Exact Top-k of the index score for a causal prefill chunk.
+
+    q (T_q, H, d) bf16, w (T_q, H) fp32, k (T_k, d) bf16, all on one CUDA
+    device; row t sits at position q_offset + t.  Returns (out_idx, out_score)
+    of shape (T_q, topk): int32 key indices and fp32 scores, sorted.
+    """
+    dev = k.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k, "k", torch.bfloat16, 2, dev)
+    T_q, H, d = q.shape
+    T_k = k.shape[0]
+    if tuple(w.shape) != (T_q, H) or k.shape[1] != d:
+        raise ValueError("shape mismatch between q (T_q,H,d), w (T_q,H) and k (T_k,d)")
+    out_idx, out_score = _outputs(T_q, topk, dev, out_idx, out_score)
+    nbytes = dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill(q.data_ptr(), w.data_ptr(), k.data_ptr(), int(q_offset), T_q,
+                                       T_k, H, d, int(topk), out_idx.data_ptr(),
+                                       out_score.data_ptr(), ws.data_ptr(), ws.numel(),
+                                       _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
+                     seq_len: torch.Tensor, topk: int, out_idx=None, out_score=None,
+                     workspace=None):
+    """Exact Top-k for one new query per sequence against its own key cache.
+
+    q (B, H, d) bf16, w (B, H) fp32, k_cache (B, t_cap, d) bf16, seq_len (B,)
+    int32 on the same device.  Returns (out_idx, out_score) of shape (B, topk).
+    """
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, 3, dev)
+    _need(seq_len, "seq_len", torch.int32, 1, dev)
+    B, H, d = q.shape
+    t_cap = k_cache.shape[1]
+    if tuple(w.shape) != (B, H) or k_cache.shape[0] != B or k_cache.shape[2] != d or seq_len.shape[0] != B:
+        raise ValueError("shape mismatch between q, w, k_cache and seq_len")
+    out_idx, out_score = _outputs(B, topk, dev, out_idx, out_score)
+    nbytes = dsa_index_decode_workspace_bytes(B, t_cap, H, d, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_decode(q.data_ptr(), w.data_ptr(), k_cache.data_ptr(),
+                                      seq_len.data_ptr(), B, t_cap, H, d, int(topk),
+                                      out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
+                                      ws.numel(), _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_device_status(workspace: torch.Tensor) -> int:
+    """Device status word of the last call that used `workspace` (synchronises)."""
+    st = ctypes.c_uint32(0)
+    with torch.cuda.device(workspace.device):
+        _check(lib().dsa_index_device_status(workspace.data_ptr(), ctypes.byref(st),
+                                             _stream_ptr(workspace.device)))
+    return int(st.value)

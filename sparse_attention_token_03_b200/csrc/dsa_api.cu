@@ -1,0 +1,314 @@
+// C ABI of libdsa_index.so: argument validation, workspace layout, TMA
+// descriptor encoding and kernel launches.  Declarations and the contract of
+// every entry point live in include/dsa_index.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/dsa_index.h"
+#include "dsa_kernels.cuh"
+
+using namespace dsa;
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DSA_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [rows][128] read as tiles of box_rows x 64 columns, 128B swizzle.
+int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DSA_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ECUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int H, int d, int topk) {
+  if (d != kD) return fail(DSA_EUNSUPPORTED, "d = %d: only d = 128 is supported", d);
+  if (H != 32 && H != 64) return fail(DSA_EUNSUPPORTED, "H = %d: only H = 32 or 64 is supported", H);
+  if (topk < 1 || topk > kMaxTopk) return fail(DSA_EUNSUPPORTED, "topk = %d outside [1, %d]", topk, kMaxTopk);
+  return DSA_OK;
+}
+
+int cap_for(int topk) {
+  int c = ((3 * topk + kTileKeys - 1) / kTileKeys) * kTileKeys;
+  return std::max(c, 3 * kTileKeys);
+}
+
+// ----------------------------------------------------------------- prefill
+struct PrefillPlan {
+  int G, n_groups, S, n_units, cap, grid;
+  size_t off_meta, off_cand, bytes;
+};
+
+PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H, int topk) {
+  PrefillPlan P{};
+  P.G = 256 / H;
+  P.n_groups = static_cast<int>((T_q + P.G - 1) / P.G);
+  const int sms = sm_count();
+  P.S = 1;
+  if (P.n_groups > 0 && P.n_groups < sms) {
+    // few long rows: split each group's keys so that every SM has work
+    const int64_t min_keys = std::max<int64_t>(q_offset_hint + 1, 1);
+    const int64_t tiles = (min_keys + kTileKeys - 1) / kTileKeys;
+    const int want = (sms + P.n_groups - 1) / P.n_groups;
+    P.S = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, tiles / 16)));
+    P.S = std::min(P.S, 64);
+  }
+  P.n_units = P.n_groups * P.S;
+  P.cap = cap_for(topk);
+  P.grid = std::max(1, std::min(sms, P.n_units));
+  size_t off = 256;  // device status word
+  P.off_meta = off;
+  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * 2 * sizeof(int32_t), 256);
+  P.off_cand = off;
+  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * 2 * P.cap * sizeof(uint64_t), 256);
+  P.bytes = off;
+  (void)T_k;
+  return P;
+}
+
+// ----------------------------------------------------------------- decode
+struct DecodePlan {
+  int grid, units_max, cap;
+  size_t off_seq_start, off_unit_tab, off_cta_ubeg, off_seq_ubeg, off_seq_ucnt, off_meta, off_cand,
+      bytes;
+};
+
+DecodePlan plan_decode(int B, int topk) {
+  DecodePlan P{};
+  P.grid = std::min(sm_count(), 1024);
+  P.units_max = P.grid + B;
+  P.cap = cap_for(topk);
+  size_t off = 256;
+  P.off_seq_start = off;
+  off = align_up(off + static_cast<size_t>(B + 1) * sizeof(int64_t), 256);
+  P.off_unit_tab = off;
+  off = align_up(off + static_cast<size_t>(P.units_max) * 3 * sizeof(int32_t), 256);
+  P.off_cta_ubeg = off;
+  off = align_up(off + static_cast<size_t>(P.grid + 1) * sizeof(int32_t), 256);
+  P.off_seq_ubeg = off;
+  off = align_up(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
+  P.off_seq_ucnt = off;
+  off = align_up(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
+  P.off_meta = off;
+  off = align_up(off + static_cast<size_t>(P.units_max) * 2 * sizeof(int32_t), 256);
+  P.off_cand = off;
+  off = align_up(off + static_cast<size_t>(P.units_max) * 2 * P.cap * sizeof(uint64_t), 256);
+  P.bytes = off;
+  return P;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_last_error_string(void) { return g_last_error.c_str(); }
+
+size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
+  if (check_shape(H, d, topk) != DSA_OK || T_q < 0 || T_k < 1) return 0;
+  // the split choice depends on q_offset; size for the most splits (q_offset = T_k - T_q)
+  return plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
+}
+
+int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                      int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
+                      float* out_score, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (T_q < 0 || T_k < 1 || q_offset < 0 || q_offset + T_q > T_k)
+    return fail(DSA_EINVAL, "need T_q >= 0, T_k >= 1, 0 <= q_offset, q_offset + T_q <= T_k");
+  if (T_k >= (int64_t(1) << 31) || T_q * H >= (int64_t(1) << 31))
+    return fail(DSA_EINVAL, "T_k and T_q*H must be below 2^31");
+  if (T_q == 0) return DSA_OK;
+  if (!q || !w || !k || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
+  const PrefillPlan P = plan_prefill(T_q, T_k, q_offset, H, topk);
+  const size_t need = plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
+  if (ws_bytes < std::max(need, P.bytes))
+    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, std::max(need, P.bytes));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUtensorMap tq, tk;
+  if ((rc = make_tmap(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+
+  ScoreParams sp{};
+  sp.mode = kModePrefill;
+  sp.topk = topk;
+  sp.cap = P.cap;
+  sp.keep_max = topk + topk / 2;
+  sp.S = P.S;
+  sp.n_groups = P.n_groups;
+  sp.n_units = P.n_units;
+  sp.q_offset = q_offset;
+  sp.T_q = T_q;
+  sp.T_k = T_k;
+  sp.w = w;
+  sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
+  sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
+  sp.err = reinterpret_cast<uint32_t*>(ws);
+  if ((e = launch_score(H, P.G, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+
+  SelectParams se{};
+  se.mode = kModePrefill;
+  se.G = P.G;
+  se.S = P.S;
+  se.topk = topk;
+  se.cap = P.cap;
+  se.n_rows = T_q;
+  se.cand = sp.cand;
+  se.meta = sp.meta;
+  se.out_idx = out_idx;
+  se.out_score = out_score;
+  se.err = sp.err;
+  if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return DSA_OK;
+}
+
+size_t dsa_index_decode_workspace_bytes(int B, int64_t t_cap, int H, int d, int topk) {
+  if (check_shape(H, d, topk) != DSA_OK || B < 1 || t_cap < 0) return 0;
+  return plan_decode(B, topk).bytes;
+}
+
+int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
+                     const int32_t* seq_len, int B, int64_t t_cap, int H, int d, int topk,
+                     int32_t* out_idx, float* out_score, void* workspace, size_t ws_bytes,
+                     void* stream) {
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (B < 1 || B > 65536 || t_cap < 0) return fail(DSA_EINVAL, "need 1 <= B <= 65536 and t_cap >= 0");
+  if (static_cast<int64_t>(B) * std::max<int64_t>(t_cap, 1) >= (int64_t(1) << 31))
+    return fail(DSA_EINVAL, "B * t_cap must be below 2^31");
+  if (!q || !w || !k_cache || !seq_len || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
+      !aligned(seq_len, 4) || !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k_cache, workspace need 16 bytes)");
+  const DecodePlan P = plan_decode(B, topk);
+  if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUtensorMap tq, tk;
+  if ((rc = make_tmap(&tq, q, static_cast<int64_t>(B) * H, H)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tk, k_cache, std::max<int64_t>(static_cast<int64_t>(B) * t_cap, 1), kTileKeys)) != DSA_OK)
+    return rc;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+
+  DecodePlanParams dp{};
+  dp.B = B;
+  dp.grid = P.grid;
+  dp.t_cap = t_cap;
+  dp.seq_len = seq_len;
+  dp.seq_start = reinterpret_cast<int64_t*>(ws + P.off_seq_start);
+  dp.unit_tab = reinterpret_cast<int32_t*>(ws + P.off_unit_tab);
+  dp.cta_ubeg = reinterpret_cast<int32_t*>(ws + P.off_cta_ubeg);
+  dp.seq_ubeg = reinterpret_cast<int32_t*>(ws + P.off_seq_ubeg);
+  dp.seq_ucnt = reinterpret_cast<int32_t*>(ws + P.off_seq_ucnt);
+  dp.err = reinterpret_cast<uint32_t*>(ws);
+  if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "decode plan launch");
+
+  ScoreParams sp{};
+  sp.mode = kModeDecode;
+  sp.topk = topk;
+  sp.cap = P.cap;
+  sp.keep_max = topk + topk / 2;
+  sp.S = 1;
+  sp.t_cap = t_cap;
+  sp.w = w;
+  sp.seq_len = seq_len;
+  sp.unit_tab = dp.unit_tab;
+  sp.cta_ubeg = dp.cta_ubeg;
+  sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
+  sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
+  sp.err = dp.err;
+  if ((e = launch_score(H, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+
+  SelectParams se{};
+  se.mode = kModeDecode;
+  se.G = 1;
+  se.S = 1;
+  se.topk = topk;
+  se.cap = P.cap;
+  se.n_rows = B;
+  se.cand = sp.cand;
+  se.meta = sp.meta;
+  se.seq_ubeg = dp.seq_ubeg;
+  se.seq_ucnt = dp.seq_ucnt;
+  se.out_idx = out_idx;
+  se.out_score = out_score;
+  se.err = dp.err;
+  if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return DSA_OK;
+}
+
+int dsa_index_device_status(const void* workspace, uint32_t* status, void* stream) {
+  if (!workspace || !status) return fail(DSA_EINVAL, "null pointer argument");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(status, workspace, 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  return DSA_OK;
+}
+
+}  // extern "C"

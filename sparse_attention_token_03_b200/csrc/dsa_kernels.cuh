@@ -1,0 +1,113 @@
+// Shared declarations of the indexer kernels: launch parameters, shared
+// memory layout and the candidate-buffer conventions.
+//
+// Candidate buffers.  A "slot" is one work unit (a query group and a range of
+// key tiles); every (slot, query) pair owns two halves of `cap` records
+// (ping-pong for compaction) and a meta pair {count, active half}.  Records
+// are 64-bit (score code << 32 | ~key): unsigned order is the selection order.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+namespace dsa {
+
+constexpr int kD = 128;          // index head width d^I (only 128 is supported)
+constexpr int kTileKeys = 128;   // keys per MMA tile (M)
+constexpr int kMaxTopk = 2048;   // largest supported k
+constexpr int kEpiThreads = 128; // epilogue warps x 32
+constexpr int kScoreThreads = 192;  // producer warp + MMA warp + 4 epilogue warps
+constexpr int kSelectThreads = 512;
+
+// Work decomposition of one fused score launch.
+enum ScoreMode : int {
+  kModePrefill = 0,  // query groups of a causal chunk; keys 0..q_offset+t
+  kModeDecode = 1,   // one query per sequence; keys 0..seq_len[b]-1 of its own cache
+  kModeGathered = 2, // query groups; keys are a gathered list (all visible), ids remapped
+};
+
+struct ScoreParams {
+  int mode;
+  int topk;
+  int cap;        // records per half-buffer
+  int keep_max;   // compaction stops refining once at most this many records remain
+  int S;          // key splits per query group (prefill / gathered)
+  int n_groups;   // query groups (prefill / gathered)
+  int n_units;    // total work units
+  int64_t q_offset;
+  int64_t T_q;
+  int64_t T_k;       // keys in the key tensor (gathered: number of gathered keys)
+  int64_t t_cap;     // decode: keys per sequence cache
+  const float* w;    // [rows][H]
+  const int32_t* seq_len;   // decode
+  const int32_t* unit_tab;  // decode: [unit][3] = {b, tile_lo, tile_hi}
+  const int32_t* cta_ubeg;  // decode: [grid + 1]
+  const int32_t* key_ids;   // gathered: real key id of each gathered key
+  uint64_t* cand;
+  int32_t* meta;
+  uint32_t* err;
+};
+
+struct SelectParams {
+  int mode;       // kModePrefill / kModeGathered: slots of row t are [(t/G)*S, +S); decode: table
+  int G;
+  int S;
+  int topk;
+  int cap;
+  int64_t n_rows;
+  const uint64_t* cand;
+  const int32_t* meta;
+  const int32_t* seq_ubeg;  // decode
+  const int32_t* seq_ucnt;  // decode
+  int32_t* out_idx;         // [n_rows][topk] (may be null when out_rec is set)
+  float* out_score;         // [n_rows][topk]
+  uint64_t* out_rec;        // optional [n_rows][topk] records (sorted, 0-padded)
+  float* out_kth;           // optional [n_rows] score of the last selected record
+  uint32_t* err;
+};
+
+struct DecodePlanParams {
+  int B;
+  int grid;
+  int64_t t_cap;
+  const int32_t* seq_len;
+  int64_t* seq_start;  // [B + 1] tile prefix
+  int32_t* unit_tab;   // [grid + B][3]
+  int32_t* cta_ubeg;   // [grid + 1]
+  int32_t* seq_ubeg;   // [B]
+  int32_t* seq_ucnt;   // [B]
+  uint32_t* err;
+};
+
+// Shared-memory footprint of the fused score kernel for N = G*H MMA columns
+// and NS key stages (host and device agree on this layout).
+struct ScoreSmem {
+  int n_cols;
+  int ns;
+  __host__ __device__ constexpr uint32_t q_sub() const { return static_cast<uint32_t>(n_cols) * 128u; }
+  __host__ __device__ constexpr uint32_t q_bytes() const { return 2u * q_sub(); }
+  __host__ __device__ constexpr uint32_t k_sub() const { return 128u * 128u; }
+  __host__ __device__ constexpr uint32_t k_stage() const { return 2u * k_sub(); }
+  __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
+  __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
+  __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + n_cols * 4u; }
+  __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + 2048u * 4u; }
+  __host__ __device__ constexpr uint32_t off_count() const { return off_thr() + 8u * 8u; }
+  __host__ __device__ constexpr uint32_t off_half() const { return off_count() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_misc() const { return off_half() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + 16u * 4u; }
+  __host__ __device__ constexpr uint32_t n_bars() const { return 2u + 2u * ns + 4u; }
+  __host__ __device__ constexpr uint32_t off_tmem() const { return off_bars() + n_bars() * 8u; }
+  __host__ __device__ constexpr uint32_t off_abort() const { return off_tmem() + 4u; }
+  __host__ __device__ constexpr uint32_t bytes() const { return off_abort() + 4u; }
+  // dynamic smem request: layout + slack to align the base to 1024 bytes
+  __host__ __device__ constexpr uint32_t request() const { return bytes() + 1024u; }
+};
+
+// Launchers (defined in the .cu files).
+cudaError_t launch_score(int H, int G, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                         const ScoreParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+cudaError_t launch_decode_plan(const DecodePlanParams& p, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,465 @@
+// Fused lightning-indexer scoring with streaming Top-k admission (sm_100a).
+//
+// Computes, for every query row t of a work unit and every visible key s,
+//     I(t,s) = sum_j w(t,j) * ReLU(q(t,j) . k(s))
+// ("DeepSeek DSA FLOPs", Lightning Indexer, eq. index score) and keeps a
+// superset of each row's Top-k in a candidate buffer, so that the T_q x T_k
+// score matrix never reaches HBM (the fused score + Top-k idea that the DoSA
+// write-up, section 04, credits to LiteTopK).
+//
+// Layout of one CTA (192 threads, one CTA per SM, persistent over units):
+//   warp 0  TMA producer: the unit's query tile once (B operand, N = G*H rows
+//           of 128 bf16), then key tiles of 128 keys (A operand) through an
+//           NS-stage ring.
+//   warp 1  TMEM owner and MMA issuer: per key tile, 8 tcgen05.mma (K = 16
+//           each) into one of two TMEM accumulators of N fp32 columns; keys
+//           sit on the 128 TMEM lanes, (query, head) on the columns.
+//   warps 2-5  epilogue: each thread owns one key (TMEM lane), reads its H
+//           dot products per query with tcgen05.ld, forms the weighted ReLU
+//           head sum in registers (heads in ascending order, fp32 FMA chain
+//           from +0), and appends (score, key) records that pass the row's
+//           running threshold.  When a row's buffer fills up, the epilogue
+//           radix-selects a new threshold and compacts the buffer.
+//
+// The admission rule keeps the selection exact: after a compaction at least
+// k records lie at or above the threshold record, so any later key below it
+// (records order by score, then smaller key first) can never enter the Top-k.
+#include "dsa_kernels.cuh"
+#include "dsa_ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Block-level helpers for the 128 epilogue threads (named barrier 1).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void epi_sync() { named_bar_sync(1, kEpiThreads); }
+
+// Warp-aggregated shared-memory histogram increment.
+__device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t digit) {
+  const uint32_t key = valid ? digit : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+  const int lane = threadIdx.x & 31;
+  if (valid && lane == (__ffs(peers) - 1)) atomicAdd(&hist[digit], __popc(peers));
+}
+
+// Find the digit bucket B holding the need-th largest record:
+// the largest B with above + sum_{d >= B} hist[d] >= need.
+// Writes {B, above + sum_{d > B} hist[d], hist[B]} to res[0..3).
+// tid in [0, 128); nb in {512, 2048}; scratch >= 4 ints.
+__device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int need, int tid,
+                                int* scratch, int* res) {
+  const int bpt = nb / kEpiThreads;
+  const int lo = tid * bpt;
+  int local = 0;
+  for (int b = 0; b < bpt; ++b) local += hist[lo + b];
+  // exclusive suffix sum over threads (higher tid = higher digits)
+  const int lane = tid & 31, wid = tid >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += v;
+  }
+  if (lane == 0) scratch[wid] = incl;  // warp total
+  epi_sync();
+  int higher_warps = 0;
+  for (int w2 = wid + 1; w2 < kEpiThreads / 32; ++w2) higher_warps += scratch[w2];
+  const int excl = incl - local + higher_warps;  // sum over threads > tid
+  if (above + excl < need && above + excl + local >= need) {
+    int acc = above + excl;
+    for (int b = bpt - 1; b >= 0; --b) {
+      const int h = hist[lo + b];
+      if (acc + h >= need) {
+        res[0] = lo + b;
+        res[1] = acc;
+        res[2] = h;
+        break;
+      }
+      acc += h;
+    }
+  }
+  epi_sync();
+}
+
+// Compact the candidate buffer of one (slot, query): keep a superset of the
+// `need` largest records that has at most keep_max records when the digits
+// allow it, raise the admission threshold to the smallest kept record prefix.
+__device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_max, int tid,
+                            uint32_t* s_hist, uint64_t* s_thr, int* s_count, int* s_half,
+                            int* s_misc) {
+  const int n = s_count[q];
+  const int half = s_half[q];
+  const uint64_t* src = buf0 + static_cast<size_t>(half) * cap;
+  uint64_t* dst = buf0 + static_cast<size_t>(half ^ 1) * cap;
+  uint64_t prefix = 0;
+  int pbits = 0, above = 0;
+  uint64_t thr = 0;
+  for (int pass = 0; pass < 6; ++pass) {
+    const int shift = max(64 - 11 * (pass + 1), 0);
+    const int width = 64 - pbits - shift;
+    const int nb = 1 << width;
+    for (int i = tid; i < nb; i += kEpiThreads) s_hist[i] = 0;
+    epi_sync();
+    for (int base = 0; base < n; base += kEpiThreads) {
+      const int i = base + tid;
+      bool ok = i < n;
+      uint64_t r = ok ? src[i] : 0ull;
+      if (pbits > 0) ok = ok && ((r >> (64 - pbits)) == prefix);
+      hist_add(s_hist, ok, static_cast<uint32_t>(r >> shift) & static_cast<uint32_t>(nb - 1));
+    }
+    epi_sync();
+    epi_find_bucket(s_hist, nb, above, need, tid, s_misc + 8, s_misc + 1);
+    const int B = s_misc[1], new_above = s_misc[2], cnt = s_misc[3];
+    prefix = (prefix << width) | static_cast<uint64_t>(B);
+    pbits += width;
+    if (new_above + cnt <= keep_max || pbits == 64) {
+      thr = (pbits == 64) ? prefix : (prefix << (64 - pbits));
+      break;
+    }
+    above = new_above;
+  }
+  if (tid == 0) s_misc[0] = 0;
+  epi_sync();
+  for (int base = 0; base < n; base += kEpiThreads) {
+    const int i = base + tid;
+    const uint64_t r = (i < n) ? src[i] : 0ull;
+    const bool keep = (i < n) && (r >= thr);
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (bal) {
+      int pos = 0;
+      const int lane = tid & 31;
+      if (lane == 0) pos = atomicAdd(&s_misc[0], __popc(bal));
+      pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+      if (keep) dst[pos + __popc(bal & lanemask_lt())] = r;
+    }
+  }
+  epi_sync();
+  if (tid == 0) {
+    s_count[q] = s_misc[0];
+    s_half[q] = half ^ 1;
+    if (thr > s_thr[q]) s_thr[q] = thr;
+  }
+  epi_sync();
+}
+
+// Geometry of one work unit, computed identically by every role.
+struct Unit {
+  int slot;         // candidate-buffer slot
+  int64_t row0;     // first query row (prefill / gathered) or sequence (decode)
+  int rows;         // valid query rows in the group
+  int64_t q_row;    // first row of the query tensor map
+  int64_t k_row;    // key tensor-map row of local key 0
+  int64_t tile_lo, tile_hi;
+  int64_t vis_base; // visible keys: local key < vis_base + row offset (prefill) or < vis_base
+};
+
+template <int G>
+__device__ __forceinline__ Unit unit_geometry(const ScoreParams& p, int u, int H) {
+  Unit U;
+  if (p.mode == kModeDecode) {
+    const int b = p.unit_tab[3 * u + 0];
+    U.slot = u;
+    U.row0 = b;
+    U.rows = 1;
+    U.q_row = static_cast<int64_t>(b) * H;
+    U.k_row = static_cast<int64_t>(b) * p.t_cap;
+    U.tile_lo = p.unit_tab[3 * u + 1];
+    U.tile_hi = p.unit_tab[3 * u + 2];
+    U.vis_base = p.seq_len[b];
+  } else {
+    const int g = p.n_groups - 1 - u / p.S;  // longest groups first
+    const int s = u % p.S;
+    U.slot = g * p.S + s;
+    U.row0 = static_cast<int64_t>(g) * G;
+    U.rows = static_cast<int>(p.T_q - U.row0 < G ? p.T_q - U.row0 : G);
+    U.q_row = U.row0 * H;
+    U.k_row = 0;
+    int64_t nkeys;
+    if (p.mode == kModePrefill) {
+      nkeys = p.q_offset + U.row0 + U.rows;  // keys visible to the group's last row
+      U.vis_base = p.q_offset + U.row0 + 1;  // row i of the group sees local keys < vis_base + i
+    } else {
+      nkeys = p.T_k;
+      U.vis_base = p.T_k;
+    }
+    const int64_t nt = (nkeys + kTileKeys - 1) / kTileKeys;
+    U.tile_lo = s * nt / p.S;
+    U.tile_hi = (s + 1) * nt / p.S;
+  }
+  return U;
+}
+
+__device__ __forceinline__ int cta_unit_begin(const ScoreParams& p) {
+  return (p.mode == kModeDecode) ? p.cta_ubeg[blockIdx.x] : static_cast<int>(blockIdx.x);
+}
+__device__ __forceinline__ int cta_unit_end(const ScoreParams& p) {
+  return (p.mode == kModeDecode) ? p.cta_ubeg[blockIdx.x + 1] : p.n_units;
+}
+__device__ __forceinline__ int cta_unit_step(const ScoreParams& p) {
+  return (p.mode == kModeDecode) ? 1 : static_cast<int>(gridDim.x);
+}
+
+}  // namespace
+
+template <int H, int G, int NS>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_topk_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
+  constexpr int N = G * H;
+  constexpr ScoreSmem L{N, NS};
+  constexpr int ACC_COLS = N;
+  constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32u : (2 * ACC_COLS <= 64) ? 64u
+                                 : (2 * ACC_COLS <= 128) ? 128u : (2 * ACC_COLS <= 256) ? 256u : 512u;
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, N);
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase;
+  const uint32_t sK = sbase + L.off_k();
+  float* s_w = reinterpret_cast<float*>(smem + L.off_w());
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + L.off_hist());
+  uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L.off_thr());
+  int* s_count = reinterpret_cast<int*>(smem + L.off_count());
+  int* s_half = reinterpret_cast<int*>(smem + L.off_half());
+  int* s_misc = reinterpret_cast<int*>(smem + L.off_misc());
+  const uint32_t bar0 = sbase + L.off_bars();
+  const uint32_t bar_q_full = bar0, bar_q_empty = bar0 + 8;
+  auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
+  auto bar_k_empty = [&](int s) { return bar0 + 16 + 8 * NS + 8 * s; };
+  auto bar_acc_full = [&](int a) { return bar0 + 16 + 16 * NS + 8 * a; };
+  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 16 * NS + 16 + 8 * a; };
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L.off_tmem());
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.off_abort());
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_acc_full(a), 1);
+      mbar_init(bar_acc_empty(a), kEpiThreads / 32);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  const int u_begin = cta_unit_begin(p), u_end = cta_unit_end(p), u_step = cta_unit_step(p);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      uint32_t kt = 0, qi = 0;
+      bool ok = true;
+      for (int u = u_begin; ok && u < u_end; u += u_step) {
+        const Unit U = unit_geometry<G>(p, u, H);
+        if (U.tile_hi <= U.tile_lo) continue;
+        if (!(ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err))) break;
+        mbar_arrive_expect_tx(bar_q_full, L.q_bytes());
+        tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
+        tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
+        ++qi;
+        for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
+          const int s = kt % NS;
+          if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err))) break;
+          mbar_arrive_expect_tx(bar_k_full(s), L.k_stage());
+          const int32_t krow = static_cast<int32_t>(U.k_row + t * kTileKeys);
+          tma_load_2d(sK + s * L.k_stage(), &tmap_k, 0, krow, bar_k_full(s));
+          tma_load_2d(sK + s * L.k_stage() + L.k_sub(), &tmap_k, 64, krow, bar_k_full(s));
+          ++kt;
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA's memory is released
+        volatile int never = 0;
+        const uint32_t first = kt > NS ? kt - NS : 0;
+        for (uint32_t i = first; i < kt; ++i)
+          mbar_wait(bar_k_full(i % NS), (i / NS) & 1, &never, p.err);
+        if (qi > 0) mbar_wait(bar_q_full, (qi - 1) & 1, &never, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t kt = 0, at = 0, qi = 0, nq = 0;
+      bool ok = true;
+      for (int u = u_begin; ok && u < u_end; u += u_step) {
+        const Unit U = unit_geometry<G>(p, u, H);
+        if (U.tile_hi <= U.tile_lo) continue;
+        if (!(ok = mbar_wait(bar_q_full, qi & 1, s_abort, p.err))) break;
+        ++qi;
+        for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
+          const int s = kt % NS;
+          const int a = at & 1;
+          if (!(ok = mbar_wait(bar_k_full(s), (kt / NS) & 1, s_abort, p.err))) break;
+          if (!(ok = mbar_wait(bar_acc_empty(a), ((at >> 1) & 1) ^ 1, s_abort, p.err))) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + a * ACC_COLS;
+          const uint32_t a_base = sK + s * L.k_stage();
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
+            const uint64_t adesc = smem_desc_sw128(a_base + sub * L.k_sub() + off);
+            const uint64_t bdesc = smem_desc_sw128(sQ + sub * L.q_sub() + off);
+            mma_bf16(d_tmem, adesc, bdesc, IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_k_empty(s));
+          mma_commit(bar_acc_full(a));
+          ++kt;
+          ++at;
+        }
+        if (ok) {
+          mma_commit(bar_q_empty);
+          ++nq;
+        }
+      }
+      // drain: make sure no MMA still writes TMEM when it is released
+      mma_commit(bar_q_empty);
+      ++nq;
+      volatile int never = 0;
+      mbar_wait(bar_q_empty, (nq - 1) & 1, &never, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int etid = threadIdx.x - 64;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = quarter * 32 + lane;
+    uint32_t at = 0;
+    bool ok = true;
+    for (int u = u_begin; ok && u < u_end; u += u_step) {
+      const Unit U = unit_geometry<G>(p, u, H);
+      epi_sync();
+      if (etid < G) {
+        s_count[etid] = 0;
+        s_thr[etid] = 0ull;
+        s_half[etid] = 0;
+      }
+      for (int i = etid; i < N; i += kEpiThreads) {
+        const int qq = i / H;
+        s_w[i] = (qq < U.rows) ? p.w[(U.row0 + qq) * H + (i % H)] : 0.0f;
+      }
+      epi_sync();
+      uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * 2 * p.cap;
+      for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
+        const int a = at & 1;
+        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
+        tc_fence_after();
+        const int64_t key_local = t * kTileKeys + row_in_tile;
+        uint32_t key_id = static_cast<uint32_t>(key_local);
+        if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
+#pragma unroll 1
+        for (int qq = 0; qq < G; ++qq) {
+          uint32_t r[H];
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                 static_cast<uint32_t>(a * ACC_COLS + qq * H);
+#pragma unroll
+          for (int c = 0; c < H / 32; ++c)
+            tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+          tmem_wait_ld();
+          const float4* w4 = reinterpret_cast<const float4*>(s_w + qq * H);
+          float acc = 0.0f;
+#pragma unroll
+          for (int j4 = 0; j4 < H / 4; ++j4) {
+            const float4 wv = w4[j4];
+            acc = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * j4 + 0]), 0.0f), acc);
+            acc = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * j4 + 1]), 0.0f), acc);
+            acc = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * j4 + 2]), 0.0f), acc);
+            acc = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * j4 + 3]), 0.0f), acc);
+          }
+          bool valid = qq < U.rows;
+          if (p.mode == kModePrefill) valid = valid && key_local < U.vis_base + qq;
+          else valid = valid && key_local < U.vis_base;
+          const uint64_t rec = make_record(acc, key_id);
+          const bool admit = valid && rec >= s_thr[qq];
+          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, admit);
+          if (bal) {
+            int pos = 0;
+            if (lane == 0) pos = atomicAdd(&s_count[qq], __popc(bal));
+            pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+            if (admit) {
+              uint64_t* buf = cand_unit + (static_cast<size_t>(qq) * 2 + s_half[qq]) * p.cap;
+              buf[pos + __popc(bal & lanemask_lt())] = rec;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_acc_empty(a));
+        ++at;
+        epi_sync();
+        for (int qq = 0; qq < G; ++qq) {
+          if (s_count[qq] > p.cap - kTileKeys)
+            epi_compact(cand_unit + static_cast<size_t>(qq) * 2 * p.cap, p.cap, qq, p.topk,
+                        p.keep_max, etid, s_hist, s_thr, s_count, s_half, s_misc);
+        }
+      }
+      if (!ok) break;
+      epi_sync();
+      if (etid < G) {
+        int32_t* m = p.meta + (static_cast<size_t>(U.slot) * G + etid) * 2;
+        m[0] = s_count[etid];
+        m[1] = s_half[etid];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launcher
+// ---------------------------------------------------------------------------
+template <int H, int G, int NS>
+static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const ScoreParams& p, int grid, cudaStream_t stream) {
+  constexpr ScoreSmem L{G * H, NS};
+  static_assert(L.request() <= 227u * 1024u, "shared memory budget");
+  auto kern = score_topk_kernel<H, G, NS>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static bool configured[64] = {};
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L.request()));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  kern<<<grid, kScoreThreads, L.request(), stream>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score(int H, int G, const CUtensorMap& tq, const CUtensorMap& tk,
+                         const ScoreParams& p, int grid, cudaStream_t stream) {
+  if (H == 64 && G == 4) return launch_score_t<64, 4, 4>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8) return launch_score_t<32, 8, 4>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 1) return launch_score_t<64, 1, 6>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 1) return launch_score_t<32, 1, 6>(tq, tk, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dsa

@@ -1,0 +1,58 @@
+"""The C ABI library loads and exports every entry point the headers declare;
+host-side argument validation answers without touching a GPU."""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import sparse_attention_token_03_b200 as dsa
+
+ROOT = Path(__file__).resolve().parent.parent
+
+
+def declared_symbols():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = h.read_text()
+        names += re.findall(r"DSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_headers_declare_the_entry_points():
+    names = set(declared_symbols())
+    for n in ("dsa_index_prefill", "dsa_index_decode", "dsa_index_prefill_workspace_bytes",
+              "dsa_index_decode_workspace_bytes", "dsa_last_error_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = dsa.lib()
+    missing = [n for n in declared_symbols() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_host_validation_without_gpu():
+    L = dsa.lib()
+    P = ctypes.c_void_p
+    dummy = P(16)
+    # unsupported head count / width / topk
+    assert L.dsa_index_prefill(dummy, dummy, dummy, 0, 4, 4, 48, 128, 8, dummy, dummy, dummy, 1 << 20, None) == -2
+    assert L.dsa_index_prefill(dummy, dummy, dummy, 0, 4, 4, 64, 64, 8, dummy, dummy, dummy, 1 << 20, None) == -2
+    assert L.dsa_index_prefill(dummy, dummy, dummy, 0, 4, 4, 64, 128, 0, dummy, dummy, dummy, 1 << 20, None) == -2
+    assert L.dsa_index_prefill(dummy, dummy, dummy, 0, 4, 4, 64, 128, 4096, dummy, dummy, dummy, 1 << 20, None) == -2
+    assert b"topk" in L.dsa_last_error_string()
+    # inconsistent sizes
+    assert L.dsa_index_prefill(dummy, dummy, dummy, 2, 4, 4, 64, 128, 8, dummy, dummy, dummy, 1 << 20, None) == -1
+    assert L.dsa_index_prefill(dummy, dummy, dummy, -1, 4, 8, 64, 128, 8, dummy, dummy, dummy, 1 << 20, None) == -1
+    # empty chunk is a no-op
+    assert L.dsa_index_prefill(None, None, dummy, 0, 0, 4, 64, 128, 8, None, None, None, 0, None) == 0
+    # null pointers
+    assert L.dsa_index_prefill(None, dummy, dummy, 0, 4, 4, 64, 128, 8, dummy, dummy, dummy, 1 << 20, None) == -1
+    # decode: bad batch
+    assert L.dsa_index_decode(dummy, dummy, dummy, dummy, 0, 16, 64, 128, 8, dummy, dummy, dummy, 1 << 20, None) == -1
+    assert L.dsa_index_decode(dummy, dummy, dummy, dummy, 4, 16, 64, 100, 8, dummy, dummy, dummy, 1 << 20, None) == -2
+    # workspace queries reject unsupported shapes with 0
+    assert L.dsa_index_prefill_workspace_bytes(4, 4, 48, 128, 8) == 0
+    assert L.dsa_index_decode_workspace_bytes(0, 16, 64, 128, 8) == 0
