@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the lightning-indexer hot path on B200.
+
+One step = one call of the library's hot path over one batch of synthetic
+input resident in HBM: for a prefill workload the fused tcgen05 score +
+streaming Top-k kernel and the final exact selection (dsa_index_prefill);
+for the decode workload the planner, the same fused kernel and the
+selection (dsa_index_decode).  The metric is causally visible (query, key)
+pairs per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
+
+Under torchrun each rank runs its own replica of the workload (different
+seed) on its own GPU; there is no collective in the data path ("scaling":
+"weak"): value = all ranks' pairs / the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from synth import WORKLOADS, make_decode, make_prefill  # noqa: E402
+
+DEFAULT_WORKLOAD = "causal_16k_h64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "sparse_attention_token_03_b200" / "csrc").glob("*")):
+        h.update(f.name.encode())
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel
+    sources have not changed since the capture (else None)."""
+    f = ROOT / "profiles" / "ncu_traffic.txt"
+    if not f.exists():
+        return None
+    cur = kernel_source_hash()
+    for line in f.read_text().splitlines():
+        parts = line.split("#", 1)[0].split()
+        if len(parts) >= 4 and parts[0] == workload and parts[1] == kernel and parts[2] == cur:
+            return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", gpu_id, "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timings (the reference arm and the cpu_baseline leg)
+# ----------------------------------------------------------------------------
+
+def oracle_sample_rate(wl, x, target_s: float, rows_cap: int | None = None):
+    """Time the oracle on evenly spaced rows; returns (pairs/s, rows, pairs, secs, cores)."""
+    import oracle
+    cores = oracle.threads()
+    if wl.kind == "decode":
+        def run(n):
+            pick = np.unique(np.linspace(0, wl.B - 1, n).round().astype(int))
+            t0 = time.perf_counter()
+            oracle.decode_topk(x["q"][pick], x["w"][pick], x["k"][pick], x["seq_len"][pick], wl.topk)
+            dt = time.perf_counter() - t0
+            return dt, int(x["seq_len"][pick].sum()), len(pick)
+        total_rows = wl.B
+    else:
+        def run(n):
+            rows = np.unique(np.linspace(0, wl.T_q - 1, n).round().astype(np.int64))
+            t0 = time.perf_counter()
+            oracle.prefill_topk(x["q"], x["w"], x["k"], x["q_offset"], wl.topk, rows=rows)
+            dt = time.perf_counter() - t0
+            return dt, int((x["q_offset"] + rows + 1).sum()), len(rows)
+        total_rows = wl.T_q
+    n = min(total_rows, max(cores, 4))
+    dt, pairs, got = run(n)
+    want = n * target_s / max(dt, 1e-3)
+    n2 = int(min(total_rows, max(n, want)))
+    if rows_cap:
+        n2 = min(n2, rows_cap)
+    if n2 > n:
+        dt, pairs, got = run(n2)
+    return pairs / dt, got, pairs, dt, cores
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = make_prefill(wl) if wl.kind == "prefill" else make_decode(wl)
+    budget = 150.0
+    per_step = budget / max(args.steps + args.warmup, 1)
+    rate, rows, pairs, dt, cores = oracle_sample_rate(wl, x, per_step)
+    # calibrated sample; now the timed steps on that sample size
+    import oracle
+    if wl.kind == "decode":
+        pick = np.unique(np.linspace(0, wl.B - 1, rows).round().astype(int))
+        step = lambda: oracle.decode_topk(x["q"][pick], x["w"][pick], x["k"][pick],
+                                          x["seq_len"][pick], wl.topk)
+        step_pairs = int(x["seq_len"][pick].sum())
+        sample = f"{len(pick)} of {wl.B} sequences per step"
+    else:
+        rws = np.unique(np.linspace(0, wl.T_q - 1, rows).round().astype(np.int64))
+        step = lambda: oracle.prefill_topk(x["q"], x["w"], x["k"], x["q_offset"], wl.topk, rows=rws)
+        step_pairs = int((x["q_offset"] + rws + 1).sum())
+        sample = f"{len(rws)} evenly spaced rows of {wl.T_q} per step ({step_pairs} pairs)"
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_pairs * args.steps / dt
+    line = {
+        "impl": "reference", "metric": "indexer causal q.k pairs/s", "value": value,
+        "unit": "pairs/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    c = {"workload": wl.name, "H": wl.H, "d": wl.d, "topk": wl.topk, "keys": wl.keys}
+    if wl.kind == "prefill":
+        c.update(T_q=wl.T_q, T_k=wl.T_k, q_offset=wl.q_offset)
+    else:
+        c.update(B=wl.B, t_cap=wl.t_cap)
+    c["pairs_per_step"] = wl.visible_pairs
+    return c
+
+
+# ----------------------------------------------------------------------------
+# CUDA arm
+# ----------------------------------------------------------------------------
+
+def main():
+    args = parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_token_03_b200 as dsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    seed = wl.seed + 7919 * rank
+    if wl.kind == "prefill":
+        x = make_prefill(wl, seed=seed)
+    else:
+        x = make_decode(wl, seed=seed)
+
+    def to_dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
+    w = torch.from_numpy(x["w"]).to(dev)
+    rows = wl.T_q if wl.kind == "prefill" else wl.B
+    out_idx = torch.empty((rows, wl.topk), dtype=torch.int32, device=dev)
+    out_score = torch.empty((rows, wl.topk), dtype=torch.float32, device=dev)
+    if wl.kind == "prefill":
+        ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(wl.T_q, wl.T_k, wl.H, wl.d, wl.topk),
+                         dtype=torch.uint8, device=dev)
+
+        def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score):
+            dsa.dsa_index_prefill(qq, ww, kk, wl.q_offset, wl.topk, out_idx=oi, out_score=osc,
+                                  workspace=ws)
+        n_kernels = 2
+    else:
+        seq_len = torch.from_numpy(x["seq_len"]).to(dev)
+        ws = torch.empty(dsa.dsa_index_decode_workspace_bytes(wl.B, wl.t_cap, wl.H, wl.d, wl.topk),
+                         dtype=torch.uint8, device=dev)
+
+        def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score, sl=seq_len):
+            dsa.dsa_index_decode(qq, ww, kk, sl, wl.topk, out_idx=oi, out_score=osc, workspace=ws)
+        n_kernels = 3
+    pairs = wl.visible_pairs
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    dsa.dsa_profile_enable(True)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize(dev)
+    if dsa.dsa_index_device_status(ws) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    step_ms, kern_ms = [], {}
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    for i in range(args.steps):
+        flush.fill_((i + 1) & 0xFF)  # evict the previous step's data from L2 (not timed)
+        ev0.record(stream)
+        step()
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms.append(ev0.elapsed_time(ev1))
+        for name, ms in dsa.dsa_profile_read():
+            kern_ms.setdefault(name, []).append(ms)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    dsa.dsa_profile_enable(False)
+    status = dsa.dsa_index_device_status(ws)
+
+    ms_step = float(np.mean(step_ms))
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = world * pairs / (ms_step * 1e-3)
+
+    # ---- roofline of the dominant kernel (the fused score + Top-k kernel)
+    pk, pk_src = peaks()
+    score_ms = float(np.mean(kern_ms.get("score_topk", [float("nan")])))
+    if wl.kind == "prefill":
+        flops = 2.0 * wl.H * wl.d * pairs
+        achieved = flops / (score_ms * 1e-3) / 1e12
+        peak = float(pk["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"bf16_tflops (burst) of {pk_src}"}
+    else:
+        nbytes = 2.0 * wl.d * pairs  # every visible key read once
+        achieved = nbytes / (score_ms * 1e-3) / 1e9
+        peak = float(pk["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"hbm_gbs of {pk_src}"}
+    roof["kernel"] = "score_topk_kernel"
+    roof["kernel_ms"] = score_ms
+    roof["traffic"] = recorded_traffic(wl.name, "score_topk_kernel")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        hk = torch.from_numpy(np.ascontiguousarray(x["k"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        hw = torch.from_numpy(x["w"]).pin_memory()
+        hoi = torch.empty(out_idx.shape, dtype=torch.int32).pin_memory()
+        hos = torch.empty(out_score.shape, dtype=torch.float32).pin_memory()
+        extra = {}
+        if wl.kind == "decode":
+            extra["sl"] = torch.from_numpy(x["seq_len"]).pin_memory()
+            dsl = torch.empty_like(seq_len)
+        dq, dk, dw = torch.empty_like(q), torch.empty_like(k), torch.empty_like(w)
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + (wl.B * 4 if wl.kind == "decode" else 0)
+        d2h = hoi.numel() * 4 + hos.numel() * 4
+        n_e2e = max(3, min(args.steps, 20))
+        e_ms = []
+        for i in range(n_e2e + 2):
+            flush.fill_(i & 0xFF)
+            ev0.record(stream)
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dw.copy_(hw, non_blocking=True)
+            if wl.kind == "decode":
+                dsl.copy_(extra["sl"], non_blocking=True)
+                step(dq, dw, dk, out_idx, out_score, dsl)
+            else:
+                step(dq, dw, dk, out_idx, out_score)
+            hoi.copy_(out_idx, non_blocking=True)
+            hos.copy_(out_score, non_blocking=True)
+            ev1.record(stream)
+            ev1.synchronize()
+            if i >= 2:
+                e_ms.append(ev0.elapsed_time(ev1))
+        em = float(np.mean(e_ms))
+        if world > 1:
+            t = torch.tensor([em], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            em = float(t.item())
+        e2e = {"value": world * pairs / (em * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": em}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, nrows, spairs, sdt, cores = oracle_sample_rate(wl, x, target_s=15.0)
+        unit = "rows" if wl.kind == "prefill" else "sequences"
+        cpu = {"value": rate, "unit": "pairs/s", "cores": cores, "kind": "oracle",
+               "sample": f"{nrows} evenly spaced {unit} of {wl.name} ({spairs} pairs, {sdt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": "indexer causal q.k pairs/s", "value": value, "unit": "pairs/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
+                                                 parallelism=f"replicas x{world}"),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": n_kernels * args.steps, "clocks": clocks, "device_status": status,
+            "kernel_ms": {n: float(np.mean(v)) for n, v in kern_ms.items()},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

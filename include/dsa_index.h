@@ -113,6 +113,18 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
  */
 DSA_API int dsa_index_device_status(const void* workspace, uint32_t* status, void* stream);
 
+/*
+ * Per-kernel timing of the calling thread's entry-point calls (for
+ * benchmarks; no counterpart on the pages).  With profiling enabled, each
+ * entry point records a CUDA event on its stream before its first kernel and
+ * after each kernel launch.  dsa_profile_read() waits for the last call's
+ * final event and returns the device time of each of its kernels in
+ * milliseconds (ms[i], names[i] may be NULL; at most max_n entries written;
+ * *n_out = number of kernels of that call).
+ */
+DSA_API int dsa_profile_enable(int on);
+DSA_API int dsa_profile_read(float* ms, const char** names, int max_n, int* n_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ from . import build as _build
 __all__ = [
     "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
-    "dsa_index_device_status",
+    "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
 ]
 
 DSA_OK = 0
@@ -60,6 +60,10 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_decode.restype = I
         L.dsa_index_device_status.argtypes = [P, P, P]
         L.dsa_index_device_status.restype = I
+        L.dsa_profile_enable.argtypes = [I]
+        L.dsa_profile_enable.restype = I
+        L.dsa_profile_read.argtypes = [P, P, I, P]
+        L.dsa_profile_read.restype = I
         _lib = L
     return _lib
 
@@ -166,6 +170,20 @@ def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
                                       out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
                                       ws.numel(), _stream_ptr(dev)))
     return out_idx, out_score
+
+
+def dsa_profile_enable(on: bool = True) -> None:
+    """Record per-kernel CUDA events inside the library's entry points."""
+    _check(lib().dsa_profile_enable(1 if on else 0))
+
+
+def dsa_profile_read() -> list[tuple[str, float]]:
+    """(kernel name, device ms) for each kernel of the calling thread's last call."""
+    ms = (ctypes.c_float * 16)()
+    names = (ctypes.c_char_p * 16)()
+    n = ctypes.c_int(0)
+    _check(lib().dsa_profile_read(ms, names, 16, ctypes.byref(n)))
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, 16))]
 
 
 def dsa_index_device_status(workspace: torch.Tensor) -> int:

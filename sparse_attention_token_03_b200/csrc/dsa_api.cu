@@ -74,6 +74,34 @@ int sm_count() {
   return n;
 }
 
+// Optional per-kernel timing: when enabled, every entry point records a CUDA
+// event on its stream before its first launch and after each launch.
+struct Profile {
+  bool enabled = false;
+  int n = 0;
+  cudaEvent_t ev[16] = {};
+  const char* name[16] = {};
+};
+thread_local Profile g_prof;
+
+void prof_begin(cudaStream_t st) {
+  if (!g_prof.enabled) return;
+  g_prof.n = 0;
+  if (!g_prof.ev[0]) cudaEventCreate(&g_prof.ev[0]);
+  cudaEventRecord(g_prof.ev[0], st);
+  g_prof.name[0] = "begin";
+  g_prof.n = 1;
+}
+
+void prof_mark(cudaStream_t st, const char* kernel) {
+  if (!g_prof.enabled || g_prof.n >= 16) return;
+  cudaEvent_t& e = g_prof.ev[g_prof.n];
+  if (!e) cudaEventCreate(&e);
+  cudaEventRecord(e, st);
+  g_prof.name[g_prof.n] = kernel;
+  ++g_prof.n;
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -191,6 +219,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
   cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  prof_begin(st);
 
   ScoreParams sp{};
   sp.mode = kModePrefill;
@@ -208,6 +237,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = reinterpret_cast<uint32_t*>(ws);
   if ((e = launch_score(H, P.G, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  prof_mark(st, "score_topk");
 
   SelectParams se{};
   se.mode = kModePrefill;
@@ -222,6 +252,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   se.out_score = out_score;
   se.err = sp.err;
   if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  prof_mark(st, "select_topk");
   return DSA_OK;
 }
 
@@ -254,6 +285,7 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
     return rc;
   cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  prof_begin(st);
 
   DecodePlanParams dp{};
   dp.B = B;
@@ -267,6 +299,7 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   dp.seq_ucnt = reinterpret_cast<int32_t*>(ws + P.off_seq_ucnt);
   dp.err = reinterpret_cast<uint32_t*>(ws);
   if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "decode plan launch");
+  prof_mark(st, "decode_plan");
 
   ScoreParams sp{};
   sp.mode = kModeDecode;
@@ -283,6 +316,7 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = dp.err;
   if ((e = launch_score(H, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  prof_mark(st, "score_topk");
 
   SelectParams se{};
   se.mode = kModeDecode;
@@ -299,6 +333,28 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   se.out_score = out_score;
   se.err = dp.err;
   if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  prof_mark(st, "select_topk");
+  return DSA_OK;
+}
+
+int dsa_profile_enable(int on) {
+  g_prof.enabled = on != 0;
+  g_prof.n = 0;
+  return DSA_OK;
+}
+
+int dsa_profile_read(float* ms, const char** names, int max_n, int* n_out) {
+  if (!ms || !n_out) return fail(DSA_EINVAL, "null pointer argument");
+  const int n = g_prof.n > 1 ? g_prof.n - 1 : 0;
+  *n_out = n;
+  if (n == 0) return DSA_OK;
+  cudaError_t e = cudaEventSynchronize(g_prof.ev[g_prof.n - 1]);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  for (int i = 0; i < n && i < max_n; ++i) {
+    e = cudaEventElapsedTime(&ms[i], g_prof.ev[i], g_prof.ev[i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    if (names) names[i] = g_prof.name[i + 1];
+  }
   return DSA_OK;
 }
 

@@ -15,8 +15,9 @@ namespace dsa {
 constexpr int kD = 128;          // index head width d^I (only 128 is supported)
 constexpr int kTileKeys = 128;   // keys per MMA tile (M)
 constexpr int kMaxTopk = 2048;   // largest supported k
-constexpr int kEpiThreads = 128; // epilogue warps x 32
-constexpr int kScoreThreads = 192;  // producer warp + MMA warp + 4 epilogue warps
+constexpr int kEpiThreads = 128; // threads of one epilogue warpgroup
+// score kernel: producer warp + MMA warp + EG epilogue warpgroups
+__host__ __device__ constexpr int score_threads(int eg) { return 64 + kEpiThreads * eg; }
 constexpr int kSelectThreads = 512;
 
 // Work decomposition of one fused score launch.
@@ -84,6 +85,7 @@ struct DecodePlanParams {
 struct ScoreSmem {
   int n_cols;
   int ns;
+  int eg;  // epilogue warpgroups (each has its own histogram and scratch)
   __host__ __device__ constexpr uint32_t q_sub() const { return static_cast<uint32_t>(n_cols) * 128u; }
   __host__ __device__ constexpr uint32_t q_bytes() const { return 2u * q_sub(); }
   __host__ __device__ constexpr uint32_t k_sub() const { return 128u * 128u; }
@@ -91,11 +93,11 @@ struct ScoreSmem {
   __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
   __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + n_cols * 4u; }
-  __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + 2048u * 4u; }
+  __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + eg * 2048u * 4u; }
   __host__ __device__ constexpr uint32_t off_count() const { return off_thr() + 8u * 8u; }
   __host__ __device__ constexpr uint32_t off_half() const { return off_count() + 8u * 4u; }
   __host__ __device__ constexpr uint32_t off_misc() const { return off_half() + 8u * 4u; }
-  __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + 16u * 4u; }
+  __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + eg * 16u * 4u; }
   __host__ __device__ constexpr uint32_t n_bars() const { return 2u + 2u * ns + 4u; }
   __host__ __device__ constexpr uint32_t off_tmem() const { return off_bars() + n_bars() * 8u; }
   __host__ __device__ constexpr uint32_t off_abort() const { return off_tmem() + 4u; }

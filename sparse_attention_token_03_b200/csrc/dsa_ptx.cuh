@@ -197,6 +197,35 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Index score of one (query, key) from its H head dot products (fp32 bit
+// patterns) and the query's head weights (16-byte aligned, shared memory):
+//     I = sum_j w_j * max(dot_j, 0)
+// in a fixed fp32 order shared by every scoring kernel of this library:
+// eight partial sums s_c (c = j mod 8), each an fp32 FMA chain over its heads
+// in ascending j starting from +0, combined as
+// ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)).
+// The eight chains give the epilogue enough independent work to issue every
+// cycle (one chain of H FMAs would stall on FMA latency).
+template <int H>
+__device__ __forceinline__ float head_sum(const uint32_t* x, const float* w) {
+  static_assert(H % 8 == 0, "H must be a multiple of 8");
+  float2 s0 = make_float2(0.0f, 0.0f), s1 = s0, s2 = s0, s3 = s0;
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+#pragma unroll
+  for (int j = 0; j < H; j += 8) {
+    const float4 wa = w4[j / 4], wb = w4[j / 4 + 1];
+    s0 = __ffma2_rn(make_float2(wa.x, wa.y),
+                    make_float2(fmaxf(__uint_as_float(x[j + 0]), 0.0f), fmaxf(__uint_as_float(x[j + 1]), 0.0f)), s0);
+    s1 = __ffma2_rn(make_float2(wa.z, wa.w),
+                    make_float2(fmaxf(__uint_as_float(x[j + 2]), 0.0f), fmaxf(__uint_as_float(x[j + 3]), 0.0f)), s1);
+    s2 = __ffma2_rn(make_float2(wb.x, wb.y),
+                    make_float2(fmaxf(__uint_as_float(x[j + 4]), 0.0f), fmaxf(__uint_as_float(x[j + 5]), 0.0f)), s2);
+    s3 = __ffma2_rn(make_float2(wb.z, wb.w),
+                    make_float2(fmaxf(__uint_as_float(x[j + 6]), 0.0f), fmaxf(__uint_as_float(x[j + 7]), 0.0f)), s3);
+  }
+  return ((s0.x + s0.y) + (s1.x + s1.y)) + ((s2.x + s2.y) + (s3.x + s3.y));
+}
+
 // Monotone 32-bit code of an fp32 score: larger score <=> larger code.
 // -0 is folded onto +0 first.
 __device__ __forceinline__ uint32_t score_code(float s) {

@@ -34,7 +34,8 @@ namespace {
 // ---------------------------------------------------------------------------
 // Block-level helpers for the 128 epilogue threads (named barrier 1).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void epi_sync() { named_bar_sync(1, kEpiThreads); }
+// Each epilogue warpgroup e synchronises on named barrier 1 + e.
+__device__ __forceinline__ void epi_sync(int bar) { named_bar_sync(bar, kEpiThreads); }
 
 // Warp-aggregated shared-memory histogram increment.
 __device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t digit) {
@@ -49,7 +50,7 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t di
 // Writes {B, above + sum_{d > B} hist[d], hist[B]} to res[0..3).
 // tid in [0, 128); nb in {512, 2048}; scratch >= 4 ints.
 __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int need, int tid,
-                                int* scratch, int* res) {
+                                int* scratch, int* res, int bar) {
   const int bpt = nb / kEpiThreads;
   const int lo = tid * bpt;
   int local = 0;
@@ -63,7 +64,7 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
     if (lane + o < 32) incl += v;
   }
   if (lane == 0) scratch[wid] = incl;  // warp total
-  epi_sync();
+  epi_sync(bar);
   int higher_warps = 0;
   for (int w2 = wid + 1; w2 < kEpiThreads / 32; ++w2) higher_warps += scratch[w2];
   const int excl = incl - local + higher_warps;  // sum over threads > tid
@@ -80,7 +81,7 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
       acc += h;
     }
   }
-  epi_sync();
+  epi_sync(bar);
 }
 
 // Compact the candidate buffer of one (slot, query): keep a superset of the
@@ -88,7 +89,7 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
 // allow it, raise the admission threshold to the smallest kept record prefix.
 __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_max, int tid,
                             uint32_t* s_hist, uint64_t* s_thr, int* s_count, int* s_half,
-                            int* s_misc) {
+                            int* s_misc, int bar) {
   const int n = s_count[q];
   const int half = s_half[q];
   const uint64_t* src = buf0 + static_cast<size_t>(half) * cap;
@@ -101,7 +102,7 @@ __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_m
     const int width = 64 - pbits - shift;
     const int nb = 1 << width;
     for (int i = tid; i < nb; i += kEpiThreads) s_hist[i] = 0;
-    epi_sync();
+    epi_sync(bar);
     for (int base = 0; base < n; base += kEpiThreads) {
       const int i = base + tid;
       bool ok = i < n;
@@ -109,8 +110,8 @@ __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_m
       if (pbits > 0) ok = ok && ((r >> (64 - pbits)) == prefix);
       hist_add(s_hist, ok, static_cast<uint32_t>(r >> shift) & static_cast<uint32_t>(nb - 1));
     }
-    epi_sync();
-    epi_find_bucket(s_hist, nb, above, need, tid, s_misc + 8, s_misc + 1);
+    epi_sync(bar);
+    epi_find_bucket(s_hist, nb, above, need, tid, s_misc + 8, s_misc + 1, bar);
     const int B = s_misc[1], new_above = s_misc[2], cnt = s_misc[3];
     prefix = (prefix << width) | static_cast<uint64_t>(B);
     pbits += width;
@@ -121,7 +122,7 @@ __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_m
     above = new_above;
   }
   if (tid == 0) s_misc[0] = 0;
-  epi_sync();
+  epi_sync(bar);
   for (int base = 0; base < n; base += kEpiThreads) {
     const int i = base + tid;
     const uint64_t r = (i < n) ? src[i] : 0ull;
@@ -135,13 +136,13 @@ __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_m
       if (keep) dst[pos + __popc(bal & lanemask_lt())] = r;
     }
   }
-  epi_sync();
+  epi_sync(bar);
   if (tid == 0) {
     s_count[q] = s_misc[0];
     s_half[q] = half ^ 1;
     if (thr > s_thr[q]) s_thr[q] = thr;
   }
-  epi_sync();
+  epi_sync(bar);
 }
 
 // Geometry of one work unit, computed identically by every role.
@@ -203,17 +204,19 @@ __device__ __forceinline__ int cta_unit_step(const ScoreParams& p) {
 
 }  // namespace
 
-template <int H, int G, int NS>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+template <int H, int G, int NS, int EG>
+__global__ void __launch_bounds__(score_threads(EG), 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
   constexpr int N = G * H;
-  constexpr ScoreSmem L{N, NS};
+  constexpr int GQ = G / EG;  // queries of a tile handled by one epilogue warpgroup
+  constexpr ScoreSmem L{N, NS, EG};
   constexpr int ACC_COLS = N;
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32u : (2 * ACC_COLS <= 64) ? 64u
                                  : (2 * ACC_COLS <= 128) ? 128u : (2 * ACC_COLS <= 256) ? 256u : 512u;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, N);
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
+  static_assert(G % EG == 0, "queries must split evenly over the epilogue warpgroups");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -222,11 +225,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const uint32_t sQ = sbase;
   const uint32_t sK = sbase + L.off_k();
   float* s_w = reinterpret_cast<float*>(smem + L.off_w());
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + L.off_hist());
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L.off_thr());
   int* s_count = reinterpret_cast<int*>(smem + L.off_count());
   int* s_half = reinterpret_cast<int*>(smem + L.off_half());
-  int* s_misc = reinterpret_cast<int*>(smem + L.off_misc());
   const uint32_t bar0 = sbase + L.off_bars();
   const uint32_t bar_q_full = bar0, bar_q_empty = bar0 + 8;
   auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_acc_full(a), 1);
-      mbar_init(bar_acc_empty(a), kEpiThreads / 32);
+      mbar_init(bar_acc_empty(a), EG * kEpiThreads / 32);
     }
     *s_abort = 0;
     fence_mbar_init();
@@ -341,24 +342,29 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int etid = threadIdx.x - 64;
+    const int e = (warp - 2) >> 2;  // epilogue warpgroup
+    const int bar = 1 + e;
+    const int etid = (threadIdx.x - 64) & (kEpiThreads - 1);
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = quarter * 32 + lane;
+    const int q_lo = e * GQ;
+    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + L.off_hist()) + e * 2048;
+    int* s_misc = reinterpret_cast<int*>(smem + L.off_misc()) + e * 16;
     uint32_t at = 0;
     bool ok = true;
     for (int u = u_begin; ok && u < u_end; u += u_step) {
       const Unit U = unit_geometry<G>(p, u, H);
-      epi_sync();
-      if (etid < G) {
-        s_count[etid] = 0;
-        s_thr[etid] = 0ull;
-        s_half[etid] = 0;
+      epi_sync(bar);
+      if (etid < GQ) {
+        s_count[q_lo + etid] = 0;
+        s_thr[q_lo + etid] = 0ull;
+        s_half[q_lo + etid] = 0;
       }
-      for (int i = etid; i < N; i += kEpiThreads) {
-        const int qq = i / H;
-        s_w[i] = (qq < U.rows) ? p.w[(U.row0 + qq) * H + (i % H)] : 0.0f;
+      for (int i = etid; i < GQ * H; i += kEpiThreads) {
+        const int qq = q_lo + i / H;
+        s_w[q_lo * H + i] = (qq < U.rows) ? p.w[(U.row0 + qq) * H + (i % H)] : 0.0f;
       }
-      epi_sync();
+      epi_sync(bar);
       uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * 2 * p.cap;
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
@@ -367,58 +373,84 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int64_t key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
-#pragma unroll 1
-        for (int qq = 0; qq < G; ++qq) {
-          uint32_t r[H];
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                 static_cast<uint32_t>(a * ACC_COLS + qq * H);
+        // per-tile copies of the admission state (only compaction changes it)
+        uint64_t thr[GQ];
+        int half[GQ];
 #pragma unroll
-          for (int c = 0; c < H / 32; ++c)
-            tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-          tmem_wait_ld();
-          const float4* w4 = reinterpret_cast<const float4*>(s_w + qq * H);
-          float acc = 0.0f;
-#pragma unroll
-          for (int j4 = 0; j4 < H / 4; ++j4) {
-            const float4 wv = w4[j4];
-            acc = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * j4 + 0]), 0.0f), acc);
-            acc = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * j4 + 1]), 0.0f), acc);
-            acc = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * j4 + 2]), 0.0f), acc);
-            acc = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * j4 + 3]), 0.0f), acc);
-          }
-          bool valid = qq < U.rows;
-          if (p.mode == kModePrefill) valid = valid && key_local < U.vis_base + qq;
-          else valid = valid && key_local < U.vis_base;
-          const uint64_t rec = make_record(acc, key_id);
-          const bool admit = valid && rec >= s_thr[qq];
-          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, admit);
-          if (bal) {
-            int pos = 0;
-            if (lane == 0) pos = atomicAdd(&s_count[qq], __popc(bal));
-            pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
-            if (admit) {
-              uint64_t* buf = cand_unit + (static_cast<size_t>(qq) * 2 + s_half[qq]) * p.cap;
-              buf[pos + __popc(bal & lanemask_lt())] = rec;
-            }
-          }
+        for (int i = 0; i < GQ; ++i) {
+          thr[i] = s_thr[q_lo + i];
+          half[i] = s_half[q_lo + i];
         }
+        // scores: TMEM loads of the next query overlap the math of this one
+        float score[GQ];
+        uint32_t r[2][H];
+        const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                              static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
+#pragma unroll
+        for (int c = 0; c < H / 32; ++c)
+          tmem_ld32(trow + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[0][c * 32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          if (i + 1 < GQ) {
+#pragma unroll
+            for (int c = 0; c < H / 32; ++c)
+              tmem_ld32(trow + (i + 1) * H + c * 32,
+                        *reinterpret_cast<uint32_t(*)[32]>(&r[(i + 1) & 1][c * 32]));
+          }
+          score[i] = head_sum<H>(r[i & 1], s_w + (q_lo + i) * H);
+          if (i + 1 < GQ) tmem_wait_ld();
+        }
+        // the accumulator can be reused as soon as it has been read
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_acc_empty(a));
         ++at;
-        epi_sync();
-        for (int qq = 0; qq < G; ++qq) {
+        // admissions of all queries, their smem reservations issued together
+        bool admit[GQ];
+        uint64_t rec[GQ];
+        uint32_t bal[GQ];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          const int qq = q_lo + i;
+          bool valid = qq < U.rows;
+          if (p.mode == kModePrefill) valid = valid && key_local < U.vis_base + qq;
+          else valid = valid && key_local < U.vis_base;
+          rec[i] = make_record(score[i], key_id);
+          admit[i] = valid && rec[i] >= thr[i];
+          bal[i] = __ballot_sync(0xFFFFFFFFu, admit[i]);
+        }
+        int pos[GQ];
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          pos[i] = 0;
+          if (lane == 0 && bal[i]) pos[i] = atomicAdd(&s_count[q_lo + i], __popc(bal[i]));
+        }
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          if (bal[i]) {
+            const int base = __shfl_sync(0xFFFFFFFFu, pos[i], 0);
+            if (admit[i]) {
+              uint64_t* buf = cand_unit + (static_cast<size_t>(q_lo + i) * 2 + half[i]) * p.cap;
+              buf[base + __popc(bal[i] & lanemask_lt())] = rec[i];
+            }
+          }
+        }
+        epi_sync(bar);
+#pragma unroll 1
+        for (int i = 0; i < GQ; ++i) {
+          const int qq = q_lo + i;
           if (s_count[qq] > p.cap - kTileKeys)
             epi_compact(cand_unit + static_cast<size_t>(qq) * 2 * p.cap, p.cap, qq, p.topk,
-                        p.keep_max, etid, s_hist, s_thr, s_count, s_half, s_misc);
+                        p.keep_max, etid, s_hist, s_thr, s_count, s_half, s_misc, bar);
         }
       }
       if (!ok) break;
-      epi_sync();
-      if (etid < G) {
-        int32_t* m = p.meta + (static_cast<size_t>(U.slot) * G + etid) * 2;
-        m[0] = s_count[etid];
-        m[1] = s_half[etid];
+      epi_sync(bar);
+      if (etid < GQ) {
+        int32_t* m = p.meta + (static_cast<size_t>(U.slot) * G + q_lo + etid) * 2;
+        m[0] = s_count[q_lo + etid];
+        m[1] = s_half[q_lo + etid];
       }
     }
   }
@@ -434,12 +466,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
-template <int H, int G, int NS>
+template <int H, int G, int NS, int EG>
 static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const ScoreParams& p, int grid, cudaStream_t stream) {
-  constexpr ScoreSmem L{G * H, NS};
+  constexpr ScoreSmem L{G * H, NS, EG};
   static_assert(L.request() <= 227u * 1024u, "shared memory budget");
-  auto kern = score_topk_kernel<H, G, NS>;
+  auto kern = score_topk_kernel<H, G, NS, EG>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool configured[64] = {};
@@ -449,16 +481,16 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  kern<<<grid, kScoreThreads, L.request(), stream>>>(tq, tk, p);
+  kern<<<grid, score_threads(EG), L.request(), stream>>>(tq, tk, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_score(int H, int G, const CUtensorMap& tq, const CUtensorMap& tk,
                          const ScoreParams& p, int grid, cudaStream_t stream) {
-  if (H == 64 && G == 4) return launch_score_t<64, 4, 4>(tq, tk, p, grid, stream);
-  if (H == 32 && G == 8) return launch_score_t<32, 8, 4>(tq, tk, p, grid, stream);
-  if (H == 64 && G == 1) return launch_score_t<64, 1, 6>(tq, tk, p, grid, stream);
-  if (H == 32 && G == 1) return launch_score_t<32, 1, 6>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 4) return launch_score_t<64, 4, 4, 2>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8) return launch_score_t<32, 8, 4, 2>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 1) return launch_score_t<64, 1, 6, 1>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 1) return launch_score_t<32, 1, 6, 1>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;
 }
 
