@@ -112,14 +112,11 @@ int check_shape(int H, int d, int topk) {
   return DSA_OK;
 }
 
-int cap_for(int topk) {
-  int c = ((3 * topk + kTileKeys - 1) / kTileKeys) * kTileKeys;
-  return std::max(c, 3 * kTileKeys);
-}
 
 // ----------------------------------------------------------------- prefill
 struct PrefillPlan {
-  int G, n_groups, S, n_units, cap, grid;
+  int G, n_groups, S, n_units, grid;
+  CandLayout lay;
   size_t off_meta, off_cand, bytes;
 };
 
@@ -138,13 +135,13 @@ PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H,
     P.S = std::min(P.S, 64);
   }
   P.n_units = P.n_groups * P.S;
-  P.cap = cap_for(topk);
+  P.lay = cand_layout(topk);
   P.grid = std::max(1, std::min(sms, P.n_units));
   size_t off = 256;  // device status word
   P.off_meta = off;
-  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * 2 * sizeof(int32_t), 256);
+  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * kMetaInts * sizeof(int32_t), 256);
   P.off_cand = off;
-  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * 2 * P.cap * sizeof(uint64_t), 256);
+  off = align_up(off + static_cast<size_t>(P.n_units) * P.G * P.lay.query_recs() * sizeof(uint64_t), 256);
   P.bytes = off;
   (void)T_k;
   return P;
@@ -152,7 +149,8 @@ PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H,
 
 // ----------------------------------------------------------------- decode
 struct DecodePlan {
-  int grid, units_max, cap;
+  int grid, units_max;
+  CandLayout lay;
   size_t off_seq_start, off_unit_tab, off_cta_ubeg, off_seq_ubeg, off_seq_ucnt, off_meta, off_cand,
       bytes;
 };
@@ -161,7 +159,7 @@ DecodePlan plan_decode(int B, int topk) {
   DecodePlan P{};
   P.grid = std::min(sm_count(), 1024);
   P.units_max = P.grid + B;
-  P.cap = cap_for(topk);
+  P.lay = cand_layout(topk);
   size_t off = 256;
   P.off_seq_start = off;
   off = align_up(off + static_cast<size_t>(B + 1) * sizeof(int64_t), 256);
@@ -174,9 +172,9 @@ DecodePlan plan_decode(int B, int topk) {
   P.off_seq_ucnt = off;
   off = align_up(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
   P.off_meta = off;
-  off = align_up(off + static_cast<size_t>(P.units_max) * 2 * sizeof(int32_t), 256);
+  off = align_up(off + static_cast<size_t>(P.units_max) * kMetaInts * sizeof(int32_t), 256);
   P.off_cand = off;
-  off = align_up(off + static_cast<size_t>(P.units_max) * 2 * P.cap * sizeof(uint64_t), 256);
+  off = align_up(off + static_cast<size_t>(P.units_max) * P.lay.query_recs() * sizeof(uint64_t), 256);
   P.bytes = off;
   return P;
 }
@@ -224,8 +222,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   ScoreParams sp{};
   sp.mode = kModePrefill;
   sp.topk = topk;
-  sp.cap = P.cap;
-  sp.keep_max = topk + topk / 2;
+  sp.lay = P.lay;
   sp.S = P.S;
   sp.n_groups = P.n_groups;
   sp.n_units = P.n_units;
@@ -244,7 +241,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   se.G = P.G;
   se.S = P.S;
   se.topk = topk;
-  se.cap = P.cap;
+  se.lay = P.lay;
   se.n_rows = T_q;
   se.cand = sp.cand;
   se.meta = sp.meta;
@@ -304,8 +301,7 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   ScoreParams sp{};
   sp.mode = kModeDecode;
   sp.topk = topk;
-  sp.cap = P.cap;
-  sp.keep_max = topk + topk / 2;
+  sp.lay = P.lay;
   sp.S = 1;
   sp.t_cap = t_cap;
   sp.w = w;
@@ -323,7 +319,7 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   se.G = 1;
   se.S = 1;
   se.topk = topk;
-  se.cap = P.cap;
+  se.lay = P.lay;
   se.n_rows = B;
   se.cand = sp.cand;
   se.meta = sp.meta;

@@ -2,9 +2,13 @@
 // memory layout and the candidate-buffer conventions.
 //
 // Candidate buffers.  A "slot" is one work unit (a query group and a range of
-// key tiles); every (slot, query) pair owns two halves of `cap` records
-// (ping-pong for compaction) and a meta pair {count, active half}.  Records
-// are 64-bit (score code << 32 | ~key): unsigned order is the selection order.
+// key tiles).  Every (slot, query) pair owns two halves (ping-pong for
+// compaction); a half holds a base region of keep_cap records (what the last
+// compaction kept) and four append regions of app_cap records, one per
+// epilogue warp (TMEM lane quarter), so that admissions need no atomics.
+// Meta per (slot, query): kMetaInts ints = {active half, base count, four
+// append counts}.  Records are 64-bit (score code << 32 | ~key): unsigned
+// order is the selection order, and 0 is never a record.
 #pragma once
 
 #include <cuda.h>
@@ -16,9 +20,35 @@ constexpr int kD = 128;          // index head width d^I (only 128 is supported)
 constexpr int kTileKeys = 128;   // keys per MMA tile (M)
 constexpr int kMaxTopk = 2048;   // largest supported k
 constexpr int kEpiThreads = 128; // threads of one epilogue warpgroup
-// score kernel: producer warp + MMA warp + EG epilogue warpgroups
-__host__ __device__ constexpr int score_threads(int eg) { return 64 + kEpiThreads * eg; }
-constexpr int kSelectThreads = 512;
+// Score kernel block: one epilogue warpgroup runs after a producer warp and an
+// MMA warp (6 warps); two epilogue warpgroups run after a whole control
+// warpgroup (producer, MMA, two idle warps) so that registers can be moved
+// between warpgroups with setmaxnreg (12 warps).
+__host__ __device__ constexpr int score_epi_warp0(int eg) { return eg == 1 ? 2 : 4; }
+__host__ __device__ constexpr int score_threads(int eg) { return 32 * score_epi_warp0(eg) + kEpiThreads * eg; }
+// Register split of the 12-warp block: 168 at launch (65536 / 384 rounded to
+// 8), then 128 x 56 (control) + 256 x 224 (epilogue) = 384 x 168.
+constexpr uint32_t kRegsLaunch12 = 168, kRegsCtl12 = 56, kRegsEpi12 = 224;
+static_assert(128 * kRegsCtl12 + 256 * kRegsEpi12 == 384 * kRegsLaunch12, "register split must balance");
+constexpr int kSelectThreads = 256;
+
+constexpr int kMetaInts = 8;
+
+struct CandLayout {
+  int keep_cap;  // records kept by a compaction (>= topk), multiple of 32
+  int app_cap;   // records per warp append region, multiple of 32
+  __host__ __device__ int half_recs() const { return keep_cap + 4 * app_cap + 32; }
+  __host__ __device__ int region_off(int r) const { return r == 0 ? 0 : keep_cap + (r - 1) * app_cap; }
+  __host__ __device__ size_t query_recs() const { return 2 * static_cast<size_t>(half_recs()); }
+};
+
+__host__ __device__ inline CandLayout cand_layout(int topk) {
+  CandLayout L;
+  L.keep_cap = ((topk + topk / 2 + 31) / 32) * 32;
+  L.app_cap = (((topk / 2 + 64) + 31) / 32) * 32;
+  if (L.app_cap < 128) L.app_cap = 128;
+  return L;
+}
 
 // Work decomposition of one fused score launch.
 enum ScoreMode : int {
@@ -30,8 +60,7 @@ enum ScoreMode : int {
 struct ScoreParams {
   int mode;
   int topk;
-  int cap;        // records per half-buffer
-  int keep_max;   // compaction stops refining once at most this many records remain
+  CandLayout lay;
   int S;          // key splits per query group (prefill / gathered)
   int n_groups;   // query groups (prefill / gathered)
   int n_units;    // total work units
@@ -54,7 +83,7 @@ struct SelectParams {
   int G;
   int S;
   int topk;
-  int cap;
+  CandLayout lay;
   int64_t n_rows;
   const uint64_t* cand;
   const int32_t* meta;
@@ -94,10 +123,12 @@ struct ScoreSmem {
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
   __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + n_cols * 4u; }
   __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + eg * 2048u * 4u; }
+  // per query: base count; per (query, warp quarter): published append count
   __host__ __device__ constexpr uint32_t off_count() const { return off_thr() + 8u * 8u; }
-  __host__ __device__ constexpr uint32_t off_half() const { return off_count() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_wcnt() const { return off_count() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_half() const { return off_wcnt() + 32u * 4u; }
   __host__ __device__ constexpr uint32_t off_misc() const { return off_half() + 8u * 4u; }
-  __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + eg * 16u * 4u; }
+  __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + eg * 32u * 4u; }
   __host__ __device__ constexpr uint32_t n_bars() const { return 2u + 2u * ns + 4u; }
   __host__ __device__ constexpr uint32_t off_tmem() const { return off_bars() + n_bars() * 8u; }
   __host__ __device__ constexpr uint32_t off_abort() const { return off_tmem() + 4u; }

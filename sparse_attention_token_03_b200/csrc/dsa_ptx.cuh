@@ -105,6 +105,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int3
       : "memory");
 }
 
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completion on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Prefetch a 2-D tile of a tensor map into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -163,6 +180,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // Shared-memory matrix descriptor for a K-major bf16 operand stored as
 // 128-byte rows with the 128B swizzle (8-row atoms of 1024 bytes).
 // byte_addr: shared address of the first row, plus the K offset inside the
@@ -186,6 +214,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Warpgroup-wide register reallocation (all 128 threads of the warpgroup).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -197,33 +235,22 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-// Index score of one (query, key) from its H head dot products (fp32 bit
-// patterns) and the query's head weights (16-byte aligned, shared memory):
+// Index score of one (query, key) from its H head dot products and the
+// query's head weights:
 //     I = sum_j w_j * max(dot_j, 0)
 // in a fixed fp32 order shared by every scoring kernel of this library:
-// eight partial sums s_c (c = j mod 8), each an fp32 FMA chain over its heads
+// eight partial sums a_c (c = j mod 8), each an fp32 FMA chain over its heads
 // in ascending j starting from +0, combined as
-// ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)).
+// ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)).
 // The eight chains give the epilogue enough independent work to issue every
-// cycle (one chain of H FMAs would stall on FMA latency).
-template <int H>
-__device__ __forceinline__ float head_sum(const uint32_t* x, const float* w) {
-  static_assert(H % 8 == 0, "H must be a multiple of 8");
-  float2 s0 = make_float2(0.0f, 0.0f), s1 = s0, s2 = s0, s3 = s0;
-  const float4* w4 = reinterpret_cast<const float4*>(w);
+// cycle (one chain of H FMAs would stall on FMA latency).  head_acc16 adds
+// 16 consecutive heads (j0 .. j0+15, j0 a multiple of 16) to the chains.
+__device__ __forceinline__ void head_acc16(float (&a)[8], const uint32_t (&x)[16], const float* w) {
 #pragma unroll
-  for (int j = 0; j < H; j += 8) {
-    const float4 wa = w4[j / 4], wb = w4[j / 4 + 1];
-    s0 = __ffma2_rn(make_float2(wa.x, wa.y),
-                    make_float2(fmaxf(__uint_as_float(x[j + 0]), 0.0f), fmaxf(__uint_as_float(x[j + 1]), 0.0f)), s0);
-    s1 = __ffma2_rn(make_float2(wa.z, wa.w),
-                    make_float2(fmaxf(__uint_as_float(x[j + 2]), 0.0f), fmaxf(__uint_as_float(x[j + 3]), 0.0f)), s1);
-    s2 = __ffma2_rn(make_float2(wb.x, wb.y),
-                    make_float2(fmaxf(__uint_as_float(x[j + 4]), 0.0f), fmaxf(__uint_as_float(x[j + 5]), 0.0f)), s2);
-    s3 = __ffma2_rn(make_float2(wb.z, wb.w),
-                    make_float2(fmaxf(__uint_as_float(x[j + 6]), 0.0f), fmaxf(__uint_as_float(x[j + 7]), 0.0f)), s3);
-  }
-  return ((s0.x + s0.y) + (s1.x + s1.y)) + ((s2.x + s2.y) + (s3.x + s3.y));
+  for (int j = 0; j < 16; ++j) a[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(x[j]), 0.0f), a[j & 7]);
+}
+__device__ __forceinline__ float head_finish(const float (&a)[8]) {
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
 // Monotone 32-bit code of an fp32 score: larger score <=> larger code.

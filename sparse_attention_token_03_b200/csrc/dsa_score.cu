@@ -84,38 +84,64 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
   epi_sync(bar);
 }
 
-// Compact the candidate buffer of one (slot, query): keep a superset of the
-// `need` largest records that has at most keep_max records when the digits
-// allow it, raise the admission threshold to the smallest kept record prefix.
-__device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_max, int tid,
-                            uint32_t* s_hist, uint64_t* s_thr, int* s_count, int* s_half,
-                            int* s_misc, int bar) {
-  const int n = s_count[q];
+// Compact the candidate buffer of one (slot, query), run by its epilogue
+// warpgroup.  The records of the active half (base region + four append
+// regions) are reduced to a superset of the `need` largest ones holding at
+// most lay.keep_cap records, written to the base region of the other half.
+// Radix digits start at the highest bit in which the smallest and largest
+// buffered records [lo, hi] differ, so one histogram pass usually decides.
+// Returns the new admission threshold (the smallest kept record prefix).
+__device__ uint64_t epi_compact(uint64_t* qbuf, const CandLayout lay, int q, int need, int tid,
+                                uint32_t* s_hist, uint64_t* s_thr, int* s_count, int* s_wcnt,
+                                int* s_half, int* s_misc, uint64_t lo, uint64_t hi, int bar) {
   const int half = s_half[q];
-  const uint64_t* src = buf0 + static_cast<size_t>(half) * cap;
-  uint64_t* dst = buf0 + static_cast<size_t>(half ^ 1) * cap;
+  const uint64_t* src = qbuf + static_cast<size_t>(half) * lay.half_recs();
+  uint64_t* dst = qbuf + static_cast<size_t>(half ^ 1) * lay.half_recs();
+  int seg_n[5];
+  seg_n[0] = s_count[q];
+#pragma unroll
+  for (int r = 1; r < 5; ++r) seg_n[r] = s_wcnt[q * 4 + r - 1];
+
   uint64_t prefix = 0;
   int pbits = 0, above = 0;
-  uint64_t thr = 0;
-  for (int pass = 0; pass < 6; ++pass) {
-    const int shift = max(64 - 11 * (pass + 1), 0);
+  const uint64_t diff = lo ^ hi;
+  if (diff != 0) {
+    pbits = __clzll(static_cast<long long>(diff));
+    prefix = pbits > 0 ? (hi >> (64 - pbits)) : 0ull;
+  }
+  uint64_t thr = lo;
+  for (int pass = 0; pass < 7 && diff != 0; ++pass) {
+    const int shift = max(64 - pbits - 11, 0);
     const int width = 64 - pbits - shift;
     const int nb = 1 << width;
     for (int i = tid; i < nb; i += kEpiThreads) s_hist[i] = 0;
     epi_sync(bar);
-    for (int base = 0; base < n; base += kEpiThreads) {
-      const int i = base + tid;
-      bool ok = i < n;
-      uint64_t r = ok ? src[i] : 0ull;
-      if (pbits > 0) ok = ok && ((r >> (64 - pbits)) == prefix);
-      hist_add(s_hist, ok, static_cast<uint32_t>(r >> shift) & static_cast<uint32_t>(nb - 1));
+#pragma unroll 1
+    for (int r = 0; r < 5; ++r) {
+      const uint64_t* sp = src + lay.region_off(r);
+      const int n = seg_n[r];
+      for (int base = 0; base < n; base += 8 * kEpiThreads) {
+        uint64_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kEpiThreads + tid;
+          v[j] = i < n ? sp[i] : 0ull;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kEpiThreads + tid;
+          bool ok = i < n;
+          if (pbits > 0) ok = ok && ((v[j] >> (64 - pbits)) == prefix);
+          hist_add(s_hist, ok, static_cast<uint32_t>(v[j] >> shift) & static_cast<uint32_t>(nb - 1));
+        }
+      }
     }
     epi_sync(bar);
-    epi_find_bucket(s_hist, nb, above, need, tid, s_misc + 8, s_misc + 1, bar);
+    epi_find_bucket(s_hist, nb, above, need, tid, s_misc + 4, s_misc + 1, bar);
     const int B = s_misc[1], new_above = s_misc[2], cnt = s_misc[3];
     prefix = (prefix << width) | static_cast<uint64_t>(B);
     pbits += width;
-    if (new_above + cnt <= keep_max || pbits == 64) {
+    if (new_above + cnt <= lay.keep_cap || pbits == 64) {
       thr = (pbits == 64) ? prefix : (prefix << (64 - pbits));
       break;
     }
@@ -123,26 +149,42 @@ __device__ void epi_compact(uint64_t* buf0, int cap, int q, int need, int keep_m
   }
   if (tid == 0) s_misc[0] = 0;
   epi_sync(bar);
-  for (int base = 0; base < n; base += kEpiThreads) {
-    const int i = base + tid;
-    const uint64_t r = (i < n) ? src[i] : 0ull;
-    const bool keep = (i < n) && (r >= thr);
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-    if (bal) {
-      int pos = 0;
-      const int lane = tid & 31;
-      if (lane == 0) pos = atomicAdd(&s_misc[0], __popc(bal));
-      pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
-      if (keep) dst[pos + __popc(bal & lanemask_lt())] = r;
+#pragma unroll 1
+  for (int r = 0; r < 5; ++r) {
+    const uint64_t* sp = src + lay.region_off(r);
+    const int n = seg_n[r];
+    for (int base = 0; base < n; base += 8 * kEpiThreads) {
+      uint64_t v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kEpiThreads + tid;
+        v[j] = i < n ? sp[i] : 0ull;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kEpiThreads + tid;
+        const bool keep = (i < n) && (v[j] >= thr);
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+        if (bal) {
+          int pos = 0;
+          if ((tid & 31) == 0) pos = atomicAdd(&s_misc[0], __popc(bal));
+          pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+          const int at = pos + __popc(bal & lanemask_lt());
+          if (keep && at < lay.keep_cap) dst[at] = v[j];
+        }
+      }
     }
   }
   epi_sync(bar);
   if (tid == 0) {
-    s_count[q] = s_misc[0];
+    s_count[q] = min(s_misc[0], lay.keep_cap);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) s_wcnt[q * 4 + r] = 0;
     s_half[q] = half ^ 1;
     if (thr > s_thr[q]) s_thr[q] = thr;
   }
   epi_sync(bar);
+  return s_thr[q];
 }
 
 // Geometry of one work unit, computed identically by every role.
@@ -265,7 +307,10 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 
   const int u_begin = cta_unit_begin(p), u_end = cta_unit_end(p), u_step = cta_unit_step(p);
 
-  if (warp == 0) {
+  if (warp < score_epi_warp0(EG)) {
+   // one setmaxnreg for the whole control warpgroup
+   if constexpr (EG == 2) regs_dec<kRegsCtl12>();
+   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
@@ -280,6 +325,11 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
         tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
         ++qi;
+        if (u + u_step < u_end) {  // warm L2 with the next unit's query tile
+          const Unit V = unit_geometry<G>(p, u + u_step, H);
+          tma_prefetch_l2_2d(&tmap_q, 0, static_cast<int32_t>(V.q_row));
+          tma_prefetch_l2_2d(&tmap_q, 64, static_cast<int32_t>(V.q_row));
+        }
         for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
           const int s = kt % NS;
           if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err))) break;
@@ -299,7 +349,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         if (qi > 0) mbar_wait(bar_q_full, (qi - 1) & 1, &never, p.err);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t kt = 0, at = 0, qi = 0, nq = 0;
@@ -340,32 +390,63 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       volatile int never = 0;
       mbar_wait(bar_q_empty, (nq - 1) & 1, &never, p.err);
     }
+   }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = (warp - 2) >> 2;  // epilogue warpgroup
+    if constexpr (EG == 2) regs_inc<kRegsEpi12>();
+    const int e = (warp - score_epi_warp0(EG)) >> 2;  // epilogue warpgroup
     const int bar = 1 + e;
-    const int etid = (threadIdx.x - 64) & (kEpiThreads - 1);
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int etid = (threadIdx.x - 32 * score_epi_warp0(EG)) & (kEpiThreads - 1);
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access = its append region
     const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lt_mask = (1u << lane) - 1u;
     const int q_lo = e * GQ;
     uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + L.off_hist()) + e * 2048;
-    int* s_misc = reinterpret_cast<int*>(smem + L.off_misc()) + e * 16;
+    int* s_misc = reinterpret_cast<int*>(smem + L.off_misc()) + e * 32;
+    uint64_t* s_wred = reinterpret_cast<uint64_t*>(s_misc + 8);  // [4] lo, [4] hi per warp
+    int* s_wcnt = reinterpret_cast<int*>(smem + L.off_wcnt());
+    const CandLayout lay = p.lay;
     uint32_t at = 0;
     bool ok = true;
     for (int u = u_begin; ok && u < u_end; u += u_step) {
       const Unit U = unit_geometry<G>(p, u, H);
       epi_sync(bar);
       if (etid < GQ) {
-        s_count[q_lo + etid] = 0;
-        s_thr[q_lo + etid] = 0ull;
-        s_half[q_lo + etid] = 0;
-      }
-      for (int i = etid; i < GQ * H; i += kEpiThreads) {
-        const int qq = q_lo + i / H;
-        s_w[q_lo * H + i] = (qq < U.rows) ? p.w[(U.row0 + qq) * H + (i % H)] : 0.0f;
+        const int qq = q_lo + etid;
+        s_count[qq] = 0;
+        s_thr[qq] = 0ull;
+        s_half[qq] = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) s_wcnt[qq * 4 + r] = 0;
       }
       epi_sync(bar);
-      uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * 2 * p.cap;
+      // this warpgroup's head weights stay in registers for the whole unit
+      float wr[GQ][H];
+#pragma unroll
+      for (int i = 0; i < GQ; ++i) {
+        const int qq = q_lo + i;
+        const float4* src = reinterpret_cast<const float4*>(p.w + (U.row0 + (qq < U.rows ? qq : 0)) * H);
+#pragma unroll
+        for (int j4 = 0; j4 < H / 4; ++j4) {
+          const float4 v = __ldg(src + j4);
+          const bool on = qq < U.rows;
+          wr[i][4 * j4 + 0] = on ? v.x : 0.0f;
+          wr[i][4 * j4 + 1] = on ? v.y : 0.0f;
+          wr[i][4 * j4 + 2] = on ? v.z : 0.0f;
+          wr[i][4 * j4 + 3] = on ? v.w : 0.0f;
+        }
+      }
+      uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * lay.query_recs();
+      // per warp and query: append count (warp-uniform); per lane: smallest
+      // and largest record it admitted (reduced only when compacting)
+      int cnt[GQ];
+      uint32_t rlo[GQ], rhi[GQ];  // score codes: records lie in [rlo << 32, (rhi << 32) | ~0]
+#pragma unroll
+      for (int i = 0; i < GQ; ++i) {
+        cnt[i] = 0;
+        rlo[i] = 0xFFFFFFFFu;
+        rhi[i] = 0u;
+      }
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
         if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
@@ -373,7 +454,6 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         const int64_t key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
-        // per-tile copies of the admission state (only compaction changes it)
         uint64_t thr[GQ];
         int half[GQ];
 #pragma unroll
@@ -381,76 +461,96 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           thr[i] = s_thr[q_lo + i];
           half[i] = s_half[q_lo + i];
         }
-        // scores: TMEM loads of the next query overlap the math of this one
-        float score[GQ];
-        uint32_t r[2][H];
+        // this warpgroup's GQ x H dot products, read in 16-column chunks: the
+        // next chunk's TMEM load overlaps the current chunk's head sums
+        constexpr int CPQ = H / 16, NC = GQ * CPQ;
         const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                               static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
-#pragma unroll
-        for (int c = 0; c < H / 32; ++c)
-          tmem_ld32(trow + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[0][c * 32]));
+        uint32_t xb[2][16];
+        float score[GQ];
+        float acc[8];
+        tmem_ld16(trow, xb[0]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < GQ; ++i) {
-          if (i + 1 < GQ) {
+        for (int c = 0; c < NC; ++c) {
+          if (c + 1 < NC) tmem_ld16(trow + (c + 1) * 16, xb[(c + 1) & 1]);
+          if (c % CPQ == 0) {
 #pragma unroll
-            for (int c = 0; c < H / 32; ++c)
-              tmem_ld32(trow + (i + 1) * H + c * 32,
-                        *reinterpret_cast<uint32_t(*)[32]>(&r[(i + 1) & 1][c * 32]));
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
           }
-          score[i] = head_sum<H>(r[i & 1], s_w + (q_lo + i) * H);
-          if (i + 1 < GQ) tmem_wait_ld();
+          head_acc16(acc, xb[c & 1], &wr[c / CPQ][(c % CPQ) * 16]);
+          if (c % CPQ == CPQ - 1) score[c / CPQ] = head_finish(acc);
+          if (c + 1 < NC) tmem_wait_ld();
+          if (c + 2 == NC || NC == 1) {
+            // every chunk has been read: the accumulator can be reused
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_acc_empty(a));
+          }
         }
-        // the accumulator can be reused as soon as it has been read
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_acc_empty(a));
         ++at;
-        // admissions of all queries, their smem reservations issued together
-        bool admit[GQ];
-        uint64_t rec[GQ];
-        uint32_t bal[GQ];
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
           bool valid = qq < U.rows;
           if (p.mode == kModePrefill) valid = valid && key_local < U.vis_base + qq;
           else valid = valid && key_local < U.vis_base;
-          rec[i] = make_record(score[i], key_id);
-          admit[i] = valid && rec[i] >= thr[i];
-          bal[i] = __ballot_sync(0xFFFFFFFFu, admit[i]);
-        }
-        int pos[GQ];
-#pragma unroll
-        for (int i = 0; i < GQ; ++i) {
-          pos[i] = 0;
-          if (lane == 0 && bal[i]) pos[i] = atomicAdd(&s_count[q_lo + i], __popc(bal[i]));
-        }
-#pragma unroll
-        for (int i = 0; i < GQ; ++i) {
-          if (bal[i]) {
-            const int base = __shfl_sync(0xFFFFFFFFu, pos[i], 0);
-            if (admit[i]) {
-              uint64_t* buf = cand_unit + (static_cast<size_t>(q_lo + i) * 2 + half[i]) * p.cap;
-              buf[base + __popc(bal[i] & lanemask_lt())] = rec[i];
-            }
+          const uint64_t rec = make_record(score[i], key_id);
+          const bool admit = valid && rec >= thr[i];
+          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, admit);
+          if (admit) {
+            uint64_t* reg = cand_unit + static_cast<size_t>(qq) * lay.query_recs() +
+                            static_cast<size_t>(half[i]) * lay.half_recs() + lay.region_off(1 + quarter);
+            reg[cnt[i] + __popc(bal & lt_mask)] = rec;
+            const uint32_t code = static_cast<uint32_t>(rec >> 32);
+            rlo[i] = min(rlo[i], code);
+            rhi[i] = max(rhi[i], code);
           }
+          cnt[i] += __popc(bal);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int i = 0; i < GQ; ++i) s_wcnt[(q_lo + i) * 4 + quarter] = cnt[i];
         }
         epi_sync(bar);
-#pragma unroll 1
+#pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
-          if (s_count[qq] > p.cap - kTileKeys)
-            epi_compact(cand_unit + static_cast<size_t>(qq) * 2 * p.cap, p.cap, qq, p.topk,
-                        p.keep_max, etid, s_hist, s_thr, s_count, s_half, s_misc, bar);
+          bool full = false;
+#pragma unroll
+          for (int w2 = 0; w2 < 4; ++w2) full = full || (s_wcnt[qq * 4 + w2] > lay.app_cap - 32);
+          if (full) {
+            // reduce the lanes' record ranges, then compact
+            uint64_t lo = static_cast<uint64_t>(__reduce_min_sync(0xFFFFFFFFu, rlo[i])) << 32;
+            uint64_t hi = (static_cast<uint64_t>(__reduce_max_sync(0xFFFFFFFFu, rhi[i])) << 32) | 0xFFFFFFFFull;
+            if (lane == 0) {
+              s_wred[quarter] = lo;
+              s_wred[4 + quarter] = hi;
+            }
+            epi_sync(bar);
+#pragma unroll
+            for (int w2 = 0; w2 < 4; ++w2) {
+              lo = s_wred[w2] < lo ? s_wred[w2] : lo;
+              hi = s_wred[4 + w2] > hi ? s_wred[4 + w2] : hi;
+            }
+            if (thr[i] > 0ull) lo = thr[i];  // every buffered record is >= the threshold
+            epi_compact(cand_unit + static_cast<size_t>(qq) * lay.query_recs(), lay, qq, p.topk, etid,
+                        s_hist, s_thr, s_count, s_wcnt, s_half, s_misc, lo, hi, bar);
+            cnt[i] = 0;
+            rlo[i] = 0xFFFFFFFFu;
+            rhi[i] = static_cast<uint32_t>(hi >> 32);
+          }
         }
       }
       if (!ok) break;
       epi_sync(bar);
       if (etid < GQ) {
-        int32_t* m = p.meta + (static_cast<size_t>(U.slot) * G + q_lo + etid) * 2;
-        m[0] = s_count[q_lo + etid];
-        m[1] = s_half[q_lo + etid];
+        const int qq = q_lo + etid;
+        int32_t* m = p.meta + (static_cast<size_t>(U.slot) * G + qq) * kMetaInts;
+        m[0] = s_half[qq];
+        m[1] = s_count[qq];
+#pragma unroll
+        for (int w2 = 0; w2 < 4; ++w2) m[2 + w2] = s_wcnt[qq * 4 + w2];
       }
     }
   }
@@ -479,6 +579,14 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L.request()));
     if (e != cudaSuccess) return e;
+    if constexpr (EG == 2) {
+      // the setmaxnreg split only balances if every thread launches with exactly
+      // kRegsLaunch12 registers; refuse to launch otherwise (it would never finish)
+      cudaFuncAttributes fa{};
+      e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != static_cast<int>(kRegsLaunch12)) return cudaErrorInvalidConfiguration;
+    }
     configured[dev] = true;
   }
   kern<<<grid, score_threads(EG), L.request(), stream>>>(tq, tk, p);

@@ -21,7 +21,8 @@ namespace dsa {
 
 namespace {
 
-template <int NT>
+constexpr int kStageRecs = 7680;  // candidates of a row staged in shared memory (60 KB)
+
 __device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_t digit) {
   const uint32_t key = valid ? digit : 0xFFFFFFFFu;
   const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
@@ -29,6 +30,7 @@ __device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_
 }
 
 // Block-wide: largest bucket B with above + sum_{d >= B} hist[d] >= need.
+// Writes {B, above + sum_{d > B} hist[d], hist[B]} to res.
 template <int NT>
 __device__ void find_bucket_blk(const uint32_t* hist, int nb, int above, int need, int* scratch,
                                 int* res) {
@@ -87,61 +89,200 @@ __device__ __forceinline__ RowUnits row_units(const SelectParams& p, int64_t row
   return r;
 }
 
+// Descending bitonic sort of 2048 records held 8 per thread (thread t owns
+// positions 8t..8t+7) by 256 threads.  Compare-exchange partners at distance
+// j < 8 sit in the same thread, 8 <= j < 256 in the same warp (register
+// shuffles), and only j >= 256 goes through shared memory.
+__device__ __forceinline__ void sort2048_desc(uint64_t (&v)[8], uint64_t* s_x) {
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int k = 2; k <= 2048; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < 8) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          if ((s & j) == 0) {
+            const int o = s | j;
+            const bool desc = (((8 * t + s) & k) == 0);
+            const uint64_t a = v[s], b = v[o];
+            const bool sw = desc ? (a < b) : (a > b);
+            v[s] = sw ? b : a;
+            v[o] = sw ? a : b;
+          }
+        }
+      } else {
+        const int m = j >> 3;
+        const bool lower = (t & m) == 0;
+        const bool desc = ((8 * t) & k) == 0;
+        const bool take_max = (lower == desc);
+        if (j < 256) {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, v[s], m);
+            v[s] = take_max ? (v[s] > o ? v[s] : o) : (v[s] < o ? v[s] : o);
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) s_x[8 * t + s] = v[s];
+          __syncthreads();
+          const int pt = t ^ m;
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint64_t o = s_x[8 * pt + s];
+            v[s] = take_max ? (v[s] > o ? v[s] : o) : (v[s] < o ? v[s] : o);
+          }
+          __syncthreads();
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
+// One CTA of 256 threads per output row.
 template <int NT>
 __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
+  static_assert(NT == 256, "the sort layout assumes 256 threads x 8 records");
+  extern __shared__ __align__(16) uint64_t s_dyn[];
+  uint64_t* s_rec = s_dyn;               // [kStageRecs] staged candidates (0 = empty slot)
+  uint64_t* s_win = s_dyn + kStageRecs;  // [2048] winners / sort exchange
   __shared__ uint32_t s_hist[2048];
-  __shared__ uint64_t s_sort[kMaxTopk];
   __shared__ int s_scratch[NT / 32];
   __shared__ int s_res[4];
-  __shared__ int s_n;
-  __shared__ int s_pos;
+  __shared__ int s_n, s_staged, s_pos;
+  __shared__ unsigned long long s_lo, s_hi;
+  __shared__ __align__(8) uint64_t s_bar;
 
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const RowUnits R = row_units(p, row);
   const int G = (p.mode == kModeDecode) ? 1 : p.G;
+  const CandLayout lay = p.lay;
+
+  // segment sg = 5 * unit + region of the row's candidate buffers
+  auto segment = [&](int sg, int& cnt) -> const uint64_t* {
+    const int u = sg / 5, r = sg % 5;
+    const size_t qi = static_cast<size_t>(R.slot_lo + u) * G + R.q;
+    const int32_t* mt = p.meta + qi * kMetaInts;
+    const int cap = (r == 0) ? lay.keep_cap : lay.app_cap;
+    cnt = min(max(mt[1 + r], 0), cap);  // counts are always in range; clamp defensively
+    return p.cand + qi * lay.query_recs() + static_cast<size_t>(mt[0] & 1) * lay.half_recs() +
+           lay.region_off(r);
+  };
+  const int n_seg = 5 * R.n_u;
 
   if (tid == 0) {
-    int n = 0;
-    for (int u = 0; u < R.n_u; ++u) {
-      const int c = p.meta[(static_cast<size_t>(R.slot_lo + u) * G + R.q) * 2];
-      n += min(max(c, 0), p.cap);
+    int n = 0, staged = 0;
+    for (int sg = 0; sg < n_seg; ++sg) {
+      int c;
+      segment(sg, c);
+      n += c;
+      staged += (c + 1) & ~1;
     }
     s_n = n;
+    s_staged = staged;
     s_pos = 0;
+    s_lo = ~0ull;
+    s_hi = 0ull;
   }
   __syncthreads();
   const int n = s_n;
   const int m = min(p.topk, n);
+  const bool staged = s_staged <= kStageRecs;
+  const int n_st = staged ? s_staged : 0;
 
-  auto unit_buf = [&](int u, int& cnt) -> const uint64_t* {
-    const int32_t* mt = p.meta + (static_cast<size_t>(R.slot_lo + u) * G + R.q) * 2;
-    cnt = min(max(mt[0], 0), p.cap);  // counts are always in range; clamp defensively
-    return p.cand + ((static_cast<size_t>(R.slot_lo + u) * G + R.q) * 2 + (mt[1] & 1)) *
-                        static_cast<size_t>(p.cap);
-  };
+  if (staged && n > 0) {
+    // one bulk copy per segment into consecutive 16-byte aligned slots
+    const uint32_t bar = smem_u32(&s_bar);
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n_st) * 8u);
+      int off = 0;
+      for (int sg = 0; sg < n_seg; ++sg) {
+        int c;
+        const uint64_t* src = segment(sg, c);
+        const int c2 = (c + 1) & ~1;
+        if (c2 > 0) bulk_load(smem_u32(s_rec + off), src, static_cast<uint32_t>(c2) * 8u, bar);
+        off += c2;
+      }
+    }
+    __syncthreads();
+    volatile int never = 0;
+    mbar_wait(bar, 0, &never, p.err);
+    __syncthreads();
+    if (tid == 0) {  // blank the padding slot after each odd-sized segment
+      int off = 0;
+      for (int sg = 0; sg < n_seg; ++sg) {
+        int c;
+        segment(sg, c);
+        if (c & 1) s_rec[off + c] = 0ull;
+        off += (c + 1) & ~1;
+      }
+    }
+    __syncthreads();
+  }
 
-  uint64_t thr = 0;  // every record is > 0, so thr = 0 keeps all
+  uint64_t thr = 1;  // records are >= 1: keeps all
   if (m > 0 && m < n) {
     uint64_t prefix = 0;
     int pbits = 0, above = 0;
-    for (int pass = 0; pass < 6; ++pass) {
-      const int shift = max(64 - 11 * (pass + 1), 0);
+    if (staged) {
+      // start the digits at the highest bit in which the records differ
+      uint64_t lo = ~0ull, hi = 0ull;
+      for (int i = tid; i < n_st; i += NT) {
+        const uint64_t r = s_rec[i];
+        if (r != 0ull) {
+          lo = r < lo ? r : lo;
+          hi = r > hi ? r : hi;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, o), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+      }
+      if ((tid & 31) == 0) {
+        atomicMin(&s_lo, static_cast<unsigned long long>(lo));
+        atomicMax(&s_hi, static_cast<unsigned long long>(hi));
+      }
+      __syncthreads();
+      const uint64_t diff = s_lo ^ s_hi;  // non-zero: records are distinct
+      pbits = __clzll(static_cast<long long>(diff));
+      prefix = pbits > 0 ? (s_hi >> (64 - pbits)) : 0ull;
+    }
+    for (int pass = 0; pass < 7; ++pass) {
+      const int shift = max(64 - pbits - 11, 0);
       const int width = 64 - pbits - shift;
       const int nb = 1 << width;
       for (int i = tid; i < nb; i += NT) s_hist[i] = 0;
       __syncthreads();
-      for (int u = 0; u < R.n_u; ++u) {
-        int cnt;
-        const uint64_t* buf = unit_buf(u, cnt);
-        for (int base = 0; base < cnt; base += NT) {
-          const int i = base + tid;
-          bool ok = i < cnt;
-          const uint64_t r = ok ? buf[i] : 0ull;
-          if (pbits > 0) ok = ok && ((r >> (64 - pbits)) == prefix);
-          hist_add_blk<NT>(s_hist, ok, static_cast<uint32_t>(r >> shift) & static_cast<uint32_t>(nb - 1));
+      auto hist_pass = [&](const uint64_t* buf, int cnt) {
+        for (int base = 0; base < cnt; base += 4 * NT) {
+          uint64_t v[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = base + j * NT + tid;
+            v[j] = i < cnt ? buf[i] : 0ull;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            bool ok = v[j] != 0ull;
+            if (pbits > 0) ok = ok && ((v[j] >> (64 - pbits)) == prefix);
+            hist_add_blk(s_hist, ok, static_cast<uint32_t>(v[j] >> shift) & static_cast<uint32_t>(nb - 1));
+          }
+        }
+      };
+      if (staged) {
+        hist_pass(s_rec, n_st);
+      } else {
+        for (int sg = 0; sg < n_seg; ++sg) {
+          int cnt;
+          const uint64_t* buf = segment(sg, cnt);
+          hist_pass(buf, cnt);
         }
       }
       __syncthreads();
@@ -158,10 +299,8 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     }
   }
 
-  // gather the winners
-  for (int u = 0; u < R.n_u; ++u) {
-    int cnt;
-    const uint64_t* buf = unit_buf(u, cnt);
+  // gather the m winners (in any order) into s_win
+  auto gather = [&](const uint64_t* buf, int cnt) {
     for (int base = 0; base < cnt; base += NT) {
       const int i = base + tid;
       const uint64_t r = (i < cnt) ? buf[i] : 0ull;
@@ -172,48 +311,62 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
         if ((tid & 31) == 0) pos = atomicAdd(&s_pos, __popc(bal));
         pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
         const int at = pos + __popc(bal & lanemask_lt());
-        if (keep && at < kMaxTopk) s_sort[at] = r;
+        if (keep && at < kMaxTopk) s_win[at] = r;
       }
+    }
+  };
+  if (staged) {
+    gather(s_rec, n_st);
+  } else {
+    for (int sg = 0; sg < n_seg; ++sg) {
+      int cnt;
+      const uint64_t* buf = segment(sg, cnt);
+      gather(buf, cnt);
     }
   }
   __syncthreads();
-  const int got = s_pos;
-  if (got != m && tid == 0) atomicOr(p.err, kErrOverflow);  // never expected
-  int P2 = 1;
-  while (P2 < m) P2 <<= 1;
-  for (int i = m + tid; i < P2; i += NT) s_sort[i] = 0ull;
-  __syncthreads();
-  // bitonic sort, descending
-  for (int k = 2; k <= P2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P2; i += NT) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t a = s_sort[i], b = s_sort[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (a < b) : (a > b)) {
-            s_sort[i] = b;
-            s_sort[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
+  if (tid == 0 && s_pos != m) atomicOr(p.err, kErrOverflow);  // never expected
+  uint64_t v[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int i = 8 * tid + s;
+    v[s] = (i < m) ? s_win[i] : 0ull;
   }
+  __syncthreads();
+  sort2048_desc(v, s_win);
   const size_t o = static_cast<size_t>(row) * p.topk;
-  for (int i = tid; i < p.topk; i += NT) {
-    const bool v = i < m;
-    const uint64_t r = v ? s_sort[i] : 0ull;
-    if (p.out_idx) p.out_idx[o + i] = v ? static_cast<int32_t>(record_key(r)) : -1;
-    if (p.out_score) p.out_score[o + i] = v ? record_score(r) : -INFINITY;
-    if (p.out_rec) p.out_rec[o + i] = r;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int i = 8 * tid + s;
+    if (i < p.topk) {
+      const bool ok = i < m;
+      if (p.out_idx) p.out_idx[o + i] = ok ? static_cast<int32_t>(record_key(v[s])) : -1;
+      if (p.out_score) p.out_score[o + i] = ok ? record_score(v[s]) : -INFINITY;
+      if (p.out_rec) p.out_rec[o + i] = ok ? v[s] : 0ull;
+    }
   }
-  if (p.out_kth && tid == 0) p.out_kth[row] = (m > 0) ? record_score(s_sort[m - 1]) : -INFINITY;
+  if (p.out_kth) {
+    if (m == 0 && tid == 0) p.out_kth[row] = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (8 * tid + s == m - 1) p.out_kth[row] = record_score(v[s]);
+  }
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   if (p.n_rows <= 0) return cudaSuccess;
-  select_topk_kernel<kSelectThreads><<<static_cast<unsigned>(p.n_rows), kSelectThreads, 0, stream>>>(p);
+  constexpr int NT = kSelectThreads;
+  const size_t smem = (kStageRecs + kMaxTopk) * sizeof(uint64_t);
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(select_topk_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  select_topk_kernel<NT><<<static_cast<unsigned>(p.n_rows), NT, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
