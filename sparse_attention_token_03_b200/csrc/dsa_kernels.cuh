@@ -45,8 +45,8 @@ struct CandLayout {
 __host__ __device__ inline CandLayout cand_layout(int topk) {
   CandLayout L;
   L.keep_cap = ((topk + topk / 2 + 31) / 32) * 32;
-  L.app_cap = (((topk / 2 + 64) + 31) / 32) * 32;
-  if (L.app_cap < 128) L.app_cap = 128;
+  L.app_cap = (((topk / 2 + 160) + 31) / 32) * 32;  // room for 4 tiles past the check threshold
+  if (L.app_cap < 256) L.app_cap = 256;
   return L;
 }
 

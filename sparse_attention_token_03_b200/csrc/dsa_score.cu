@@ -466,23 +466,25 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         constexpr int CPQ = H / 16, NC = GQ * CPQ;
         const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                               static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
-        uint32_t xb[2][16];
+        uint32_t xb[3][16];
         float score[GQ];
         float acc[8];
         tmem_ld16(trow, xb[0]);
+        if (NC > 1) tmem_ld16(trow + 16, xb[1]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-          if (c + 1 < NC) tmem_ld16(trow + (c + 1) * 16, xb[(c + 1) & 1]);
+          // loads run two chunks ahead of the math
+          if (c + 2 < NC) tmem_ld16(trow + (c + 2) * 16, xb[(c + 2) % 3]);
           if (c % CPQ == 0) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
           }
-          head_acc16(acc, xb[c & 1], &wr[c / CPQ][(c % CPQ) * 16]);
+          head_acc16(acc, xb[c % 3], &wr[c / CPQ][(c % CPQ) * 16]);
           if (c % CPQ == CPQ - 1) score[c / CPQ] = head_finish(acc);
-          if (c + 1 < NC) tmem_wait_ld();
-          if (c + 2 == NC || NC == 1) {
-            // every chunk has been read: the accumulator can be reused
+          if (c + 2 < NC) tmem_wait_ld();
+          // after the last load has landed, release the accumulator
+          if ((NC <= 2 && c == 0) || (NC > 2 && c + 3 == NC)) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_acc_empty(a));
@@ -508,6 +510,10 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           }
           cnt[i] += __popc(bal);
         }
+        // every 4th tile (and at the unit's end) the warpgroup publishes its
+        // append counts and compacts the buffers that could overflow within
+        // the next 4 tiles (a warp appends at most 32 records per query per tile)
+        if (((t - U.tile_lo) & 3) != 3 && t + 1 != U.tile_hi) continue;
         if (lane == 0) {
 #pragma unroll
           for (int i = 0; i < GQ; ++i) s_wcnt[(q_lo + i) * 4 + quarter] = cnt[i];
@@ -518,7 +524,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           const int qq = q_lo + i;
           bool full = false;
 #pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) full = full || (s_wcnt[qq * 4 + w2] > lay.app_cap - 32);
+          for (int w2 = 0; w2 < 4; ++w2) full = full || (s_wcnt[qq * 4 + w2] > lay.app_cap - 4 * 32);
           if (full) {
             // reduce the lanes' record ranges, then compact
             uint64_t lo = static_cast<uint64_t>(__reduce_min_sync(0xFFFFFFFFu, rlo[i])) << 32;
