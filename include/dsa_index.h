@@ -106,6 +106,32 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
                      void* stream);
 
 /*
+ * Batched decode that allocates nothing (no counterpart in the paper; a
+ * library convenience).  Same computation, arguments and outputs as
+ * dsa_index_decode, without the workspace: for callers that cannot hand the
+ * library device memory of their own, such as hosts whose device memory is
+ * entirely carved up by an allocator they do not control, or code that must
+ * not call cudaMalloc on a latency-critical path because it can synchronise
+ * the device.
+ *  - Scratch is a fixed array in the library's device image, sized for at
+ *    most 64 sequences at topk <= 2048 (about 28 MB).  Every GPU on which the
+ *    library is loaded holds that memory until the process exits.  B > 64
+ *    returns DSA_EINVAL with an explanatory message; nothing is launched.
+ *  - The call itself allocates no device memory: no cudaMalloc/cudaFree, no
+ *    allocating library routine.  The first call on each device looks up the
+ *    scratch's device address (with that device current); make that first
+ *    call before any stream capture.
+ *  - All calls share the one scratch array, which keeps the last call's
+ *    contents; each call initialises what it reads.  Calls whose executions
+ *    overlap on the GPU (different streams, or host threads racing on the
+ *    same device) race on the scratch and give undefined results: serialise
+ *    them.
+ */
+DSA_API int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const uint16_t* k_cache,
+                                     const int32_t* seq_len, int B, int64_t t_cap, int H, int d,
+                                     int topk, int32_t* out_idx, float* out_score, void* stream);
+
+/*
  * Device status word of the most recent call that used `workspace`: 0 when
  * every device-side check passed.  Synchronises `stream`.
  * Bit 0: a bounded wait inside a kernel gave up (the kernel unwound).

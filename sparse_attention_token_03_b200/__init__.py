@@ -20,6 +20,7 @@ __all__ = [
     "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
+    "dsa_index_decode_noalloc",
 ]
 
 DSA_OK = 0
@@ -58,6 +59,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_decode_workspace_bytes.restype = SZ
         L.dsa_index_decode.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]
         L.dsa_index_decode.restype = I
+        L.dsa_index_decode_noalloc.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P]
+        L.dsa_index_decode_noalloc.restype = I
         L.dsa_index_device_status.argtypes = [P, P, P]
         L.dsa_index_device_status.restype = I
         L.dsa_profile_enable.argtypes = [I]
@@ -169,6 +172,29 @@ def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
                                       seq_len.data_ptr(), B, t_cap, H, d, int(topk),
                                       out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
                                       ws.numel(), _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_decode_noalloc(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
+                             seq_len: torch.Tensor, topk: int, out_idx=None, out_score=None):
+    """dsa_index_decode without a workspace: the library's static device
+    scratch serves at most 64 sequences, and calls must not overlap on the GPU.
+    Pass preallocated outputs to keep the call free of any allocation."""
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, 3, dev)
+    _need(seq_len, "seq_len", torch.int32, 1, dev)
+    B, H, d = q.shape
+    t_cap = k_cache.shape[1]
+    if tuple(w.shape) != (B, H) or k_cache.shape[0] != B or k_cache.shape[2] != d or seq_len.shape[0] != B:
+        raise ValueError("shape mismatch between q, w, k_cache and seq_len")
+    out_idx, out_score = _outputs(B, topk, dev, out_idx, out_score)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_decode_noalloc(q.data_ptr(), w.data_ptr(), k_cache.data_ptr(),
+                                              seq_len.data_ptr(), B, t_cap, H, d, int(topk),
+                                              out_idx.data_ptr(), out_score.data_ptr(),
+                                              _stream_ptr(dev)))
     return out_idx, out_score
 
 

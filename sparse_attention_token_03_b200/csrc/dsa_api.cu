@@ -155,28 +155,146 @@ struct DecodePlan {
       bytes;
 };
 
-DecodePlan plan_decode(int B, int topk) {
+constexpr size_t align_c(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout of a batched decode of B sequences run on `grid` CTAs.
+constexpr DecodePlan plan_decode_layout(int B, int topk, int grid) {
   DecodePlan P{};
-  P.grid = std::min(sm_count(), 1024);
+  P.grid = grid;
   P.units_max = P.grid + B;
   P.lay = cand_layout(topk);
   size_t off = 256;
   P.off_seq_start = off;
-  off = align_up(off + static_cast<size_t>(B + 1) * sizeof(int64_t), 256);
+  off = align_c(off + static_cast<size_t>(B + 1) * sizeof(int64_t), 256);
   P.off_unit_tab = off;
-  off = align_up(off + static_cast<size_t>(P.units_max) * 3 * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(P.units_max) * 3 * sizeof(int32_t), 256);
   P.off_cta_ubeg = off;
-  off = align_up(off + static_cast<size_t>(P.grid + 1) * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(P.grid + 1) * sizeof(int32_t), 256);
   P.off_seq_ubeg = off;
-  off = align_up(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
   P.off_seq_ucnt = off;
-  off = align_up(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
   P.off_meta = off;
-  off = align_up(off + static_cast<size_t>(P.units_max) * kMetaInts * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(P.units_max) * kMetaInts * sizeof(int32_t), 256);
   P.off_cand = off;
-  off = align_up(off + static_cast<size_t>(P.units_max) * P.lay.query_recs() * sizeof(uint64_t), 256);
+  off = align_c(off + static_cast<size_t>(P.units_max) * P.lay.query_recs() * sizeof(uint64_t), 256);
   P.bytes = off;
   return P;
+}
+
+DecodePlan plan_decode(int B, int topk) { return plan_decode_layout(B, topk, std::min(sm_count(), 1024)); }
+
+int check_decode_args(const uint16_t* q, const float* w, const uint16_t* k_cache,
+                      const int32_t* seq_len, int B, int64_t t_cap, int H, int d, int topk,
+                      int32_t* out_idx, float* out_score) {
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (B < 1 || B > 65536 || t_cap < 0) return fail(DSA_EINVAL, "need 1 <= B <= 65536 and t_cap >= 0");
+  if (static_cast<int64_t>(B) * std::max<int64_t>(t_cap, 1) >= (int64_t(1) << 31))
+    return fail(DSA_EINVAL, "B * t_cap must be below 2^31");
+  if (!q || !w || !k_cache || !seq_len || !out_idx || !out_score)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(w, 4) || !aligned(seq_len, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q and k_cache need 16 bytes)");
+  return DSA_OK;
+}
+
+// The decode path proper (arguments already validated): planner, fused score
+// kernel and final selection, all on `st`, scratch in `ws` laid out by P.
+int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const int32_t* seq_len,
+               int B, int64_t t_cap, int H, int topk, int32_t* out_idx, float* out_score,
+               uint8_t* ws, const DecodePlan& P, bool profile, cudaStream_t st) {
+  int rc;
+  CUtensorMap tq, tk;
+  if ((rc = make_tmap(&tq, q, static_cast<int64_t>(B) * H, H)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tk, k_cache, std::max<int64_t>(static_cast<int64_t>(B) * t_cap, 1), kTileKeys)) != DSA_OK)
+    return rc;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (profile) prof_begin(st);
+
+  DecodePlanParams dp{};
+  dp.B = B;
+  dp.grid = P.grid;
+  dp.t_cap = t_cap;
+  dp.seq_len = seq_len;
+  dp.seq_start = reinterpret_cast<int64_t*>(ws + P.off_seq_start);
+  dp.unit_tab = reinterpret_cast<int32_t*>(ws + P.off_unit_tab);
+  dp.cta_ubeg = reinterpret_cast<int32_t*>(ws + P.off_cta_ubeg);
+  dp.seq_ubeg = reinterpret_cast<int32_t*>(ws + P.off_seq_ubeg);
+  dp.seq_ucnt = reinterpret_cast<int32_t*>(ws + P.off_seq_ucnt);
+  dp.err = reinterpret_cast<uint32_t*>(ws);
+  if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "decode plan launch");
+  if (profile) prof_mark(st, "decode_plan");
+
+  ScoreParams sp{};
+  sp.mode = kModeDecode;
+  sp.topk = topk;
+  sp.lay = P.lay;
+  sp.S = 1;
+  sp.t_cap = t_cap;
+  sp.w = w;
+  sp.seq_len = seq_len;
+  sp.unit_tab = dp.unit_tab;
+  sp.cta_ubeg = dp.cta_ubeg;
+  sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
+  sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
+  sp.err = dp.err;
+  if ((e = launch_score(H, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  if (profile) prof_mark(st, "score_topk");
+
+  SelectParams se{};
+  se.mode = kModeDecode;
+  se.G = 1;
+  se.S = 1;
+  se.topk = topk;
+  se.lay = P.lay;
+  se.n_rows = B;
+  se.cand = sp.cand;
+  se.meta = sp.meta;
+  se.seq_ubeg = dp.seq_ubeg;
+  se.seq_ucnt = dp.seq_ucnt;
+  se.out_idx = out_idx;
+  se.out_score = out_score;
+  se.err = dp.err;
+  if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  if (profile) prof_mark(st, "select_topk");
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Scratch for dsa_index_decode_noalloc.  The array lives in the library's
+// device image, so every GPU on which the library's kernels are loaded holds
+// it (about 28 MB) until the process exits.  Host code must not hand the
+// symbol itself to a kernel: on the host it only names a stand-in; the device
+// address comes from cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+constexpr int kNoAllocMaxB = 64;      // largest batch served from the static scratch
+constexpr int kNoAllocMaxGrid = 160;  // persistent CTAs used by that path (<= SMs)
+constexpr size_t kNoAllocScratchBytes = plan_decode_layout(kNoAllocMaxB, kMaxTopk, kNoAllocMaxGrid).bytes;
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the static scratch on the current device (looked up on
+// the first call per device, with that device current).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(DSA_EUNSUPPORTED, "device index %d above 63", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
 }
 
 }  // namespace
@@ -262,75 +380,33 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
                      const int32_t* seq_len, int B, int64_t t_cap, int H, int d, int topk,
                      int32_t* out_idx, float* out_score, void* workspace, size_t ws_bytes,
                      void* stream) {
-  int rc = check_shape(H, d, topk);
+  int rc = check_decode_args(q, w, k_cache, seq_len, B, t_cap, H, d, topk, out_idx, out_score);
   if (rc != DSA_OK) return rc;
-  if (B < 1 || B > 65536 || t_cap < 0) return fail(DSA_EINVAL, "need 1 <= B <= 65536 and t_cap >= 0");
-  if (static_cast<int64_t>(B) * std::max<int64_t>(t_cap, 1) >= (int64_t(1) << 31))
-    return fail(DSA_EINVAL, "B * t_cap must be below 2^31");
-  if (!q || !w || !k_cache || !seq_len || !out_idx || !out_score || !workspace)
-    return fail(DSA_EINVAL, "null pointer argument");
-  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
-      !aligned(seq_len, 4) || !aligned(out_idx, 4) || !aligned(out_score, 4))
-    return fail(DSA_EINVAL, "misaligned pointer (q, k_cache, workspace need 16 bytes)");
+  if (!workspace) return fail(DSA_EINVAL, "null workspace");
+  if (!aligned(workspace, 16)) return fail(DSA_EINVAL, "misaligned workspace (needs 16 bytes)");
   const DecodePlan P = plan_decode(B, topk);
   if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  CUtensorMap tq, tk;
-  if ((rc = make_tmap(&tq, q, static_cast<int64_t>(B) * H, H)) != DSA_OK) return rc;
-  if ((rc = make_tmap(&tk, k_cache, std::max<int64_t>(static_cast<int64_t>(B) * t_cap, 1), kTileKeys)) != DSA_OK)
-    return rc;
-  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  prof_begin(st);
+  return decode_run(q, w, k_cache, seq_len, B, t_cap, H, topk, out_idx, out_score,
+                    static_cast<uint8_t*>(workspace), P, true, static_cast<cudaStream_t>(stream));
+}
 
-  DecodePlanParams dp{};
-  dp.B = B;
-  dp.grid = P.grid;
-  dp.t_cap = t_cap;
-  dp.seq_len = seq_len;
-  dp.seq_start = reinterpret_cast<int64_t*>(ws + P.off_seq_start);
-  dp.unit_tab = reinterpret_cast<int32_t*>(ws + P.off_unit_tab);
-  dp.cta_ubeg = reinterpret_cast<int32_t*>(ws + P.off_cta_ubeg);
-  dp.seq_ubeg = reinterpret_cast<int32_t*>(ws + P.off_seq_ubeg);
-  dp.seq_ucnt = reinterpret_cast<int32_t*>(ws + P.off_seq_ucnt);
-  dp.err = reinterpret_cast<uint32_t*>(ws);
-  if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "decode plan launch");
-  prof_mark(st, "decode_plan");
-
-  ScoreParams sp{};
-  sp.mode = kModeDecode;
-  sp.topk = topk;
-  sp.lay = P.lay;
-  sp.S = 1;
-  sp.t_cap = t_cap;
-  sp.w = w;
-  sp.seq_len = seq_len;
-  sp.unit_tab = dp.unit_tab;
-  sp.cta_ubeg = dp.cta_ubeg;
-  sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
-  sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
-  sp.err = dp.err;
-  if ((e = launch_score(H, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
-  prof_mark(st, "score_topk");
-
-  SelectParams se{};
-  se.mode = kModeDecode;
-  se.G = 1;
-  se.S = 1;
-  se.topk = topk;
-  se.lay = P.lay;
-  se.n_rows = B;
-  se.cand = sp.cand;
-  se.meta = sp.meta;
-  se.seq_ubeg = dp.seq_ubeg;
-  se.seq_ucnt = dp.seq_ucnt;
-  se.out_idx = out_idx;
-  se.out_score = out_score;
-  se.err = dp.err;
-  if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
-  prof_mark(st, "select_topk");
-  return DSA_OK;
+int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const uint16_t* k_cache,
+                             const int32_t* seq_len, int B, int64_t t_cap, int H, int d, int topk,
+                             int32_t* out_idx, float* out_score, void* stream) {
+  int rc = check_decode_args(q, w, k_cache, seq_len, B, t_cap, H, d, topk, out_idx, out_score);
+  if (rc != DSA_OK) return rc;
+  if (B > kNoAllocMaxB)
+    return fail(DSA_EINVAL,
+                "dsa_index_decode_noalloc: B = %d sequences exceeds the static scratch limit of %d; "
+                "use dsa_index_decode with a caller workspace",
+                B, kNoAllocMaxB);
+  const DecodePlan P = plan_decode_layout(B, topk, std::min(sm_count(), kNoAllocMaxGrid));
+  if (P.bytes > kNoAllocScratchBytes)
+    return fail(DSA_EWORKSPACE, "static decode scratch of %zu bytes, %zu needed", kNoAllocScratchBytes, P.bytes);
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws)) != DSA_OK) return rc;
+  return decode_run(q, w, k_cache, seq_len, B, t_cap, H, topk, out_idx, out_score,
+                    static_cast<uint8_t*>(ws), P, false, static_cast<cudaStream_t>(stream));
 }
 
 int dsa_profile_enable(int on) {

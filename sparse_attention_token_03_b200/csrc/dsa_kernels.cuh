@@ -37,13 +37,13 @@ constexpr int kMetaInts = 8;
 struct CandLayout {
   int keep_cap;  // records kept by a compaction (>= topk), multiple of 32
   int app_cap;   // records per warp append region, multiple of 32
-  __host__ __device__ int half_recs() const { return keep_cap + 4 * app_cap + 32; }
-  __host__ __device__ int region_off(int r) const { return r == 0 ? 0 : keep_cap + (r - 1) * app_cap; }
-  __host__ __device__ size_t query_recs() const { return 2 * static_cast<size_t>(half_recs()); }
+  __host__ __device__ constexpr int half_recs() const { return keep_cap + 4 * app_cap + 32; }
+  __host__ __device__ constexpr int region_off(int r) const { return r == 0 ? 0 : keep_cap + (r - 1) * app_cap; }
+  __host__ __device__ constexpr size_t query_recs() const { return 2 * static_cast<size_t>(half_recs()); }
 };
 
-__host__ __device__ inline CandLayout cand_layout(int topk) {
-  CandLayout L;
+__host__ __device__ constexpr CandLayout cand_layout(int topk) {
+  CandLayout L{0, 0};
   L.keep_cap = ((topk + topk / 2 + 31) / 32) * 32;
   L.app_cap = (((topk / 2 + 160) + 31) / 32) * 32;  // room for 4 tiles past the check threshold
   if (L.app_cap < 256) L.app_cap = 256;
