@@ -106,6 +106,42 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
                      void* stream);
 
 /*
+ * Chunked causal prefill with DoSA certified pruning ("DoSA: Dots Sparse
+ * Attention", steps 1-3; 163.com write-up, section 03).  Same inputs and the
+ * same outputs, bit for bit, as dsa_index_prefill: the seed set only changes
+ * how much work is skipped, never the result.
+ *   1. The n_seed seed keys are scored with all heads; per row, tau is the
+ *      topk-th largest seed score (a lower bound on the row's true topk-th).
+ *   2. Every other visible key gets an upper bound U from 14 retained heads,
+ *      a residual bound for the omitted positive-weight heads and a folded
+ *      lower bound on the omitted negative-weight heads' penalty; keys with
+ *      U < tau are pruned (strictly; a key whose bound is uncertain is kept).
+ *   3. Survivors are scored exactly with all heads; records at or above the
+ *      row's topk-th seed record enter the final exact Top-k with the seeds'.
+ *   seed_idx   device, [n_seed] int32: distinct keys with 0 <= seed < q_offset
+ *              (visible to every row); topk <= n_seed <= q_offset, else
+ *              DSA_ESEED before any launch.  Out-of-range or repeated seeds
+ *              found on the device make every row fall back to the exact
+ *              dense computation (reported as DSA_ESEED when stats is given).
+ *   stats      host, may be NULL: when given, the call synchronises `stream`
+ *              and fills the counters (screened_pairs: visible non-seed
+ *              pairs; survivor_pairs: pairs with U >= tau; refined_pairs:
+ *              survivors scored exactly; records: seed Top-k + refined
+ *              records; recovered_rows: rows recomputed densely because
+ *              their survivors exceeded the per-row list capacity of
+ *              max(T_k / 4, 4 topk) keys).
+ * Requires T_q <= 65536.  The workspace is sized by
+ * dsa_index_prefill_pruned_workspace_bytes().
+ */
+DSA_API size_t dsa_index_prefill_pruned_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                                        int n_seed);
+DSA_API int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                                     int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                     const int32_t* seed_idx, int n_seed, int32_t* out_idx,
+                                     float* out_score, dsa_stats* stats, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
+/*
  * Batched decode that allocates nothing (no counterpart in the paper; a
  * library convenience).  Same computation, arguments and outputs as
  * dsa_index_decode, without the workspace: for callers that cannot hand the

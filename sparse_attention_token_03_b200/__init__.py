@@ -20,7 +20,7 @@ __all__ = [
     "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
-    "dsa_index_decode_noalloc",
+    "dsa_index_decode_noalloc", "dsa_index_prefill_pruned", "dsa_index_prefill_pruned_workspace_bytes",
 ]
 
 DSA_OK = 0
@@ -59,6 +59,10 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_decode_workspace_bytes.restype = SZ
         L.dsa_index_decode.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]
         L.dsa_index_decode.restype = I
+        L.dsa_index_prefill_pruned_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
+        L.dsa_index_prefill_pruned_workspace_bytes.restype = SZ
+        L.dsa_index_prefill_pruned.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I, P, P, P, P, SZ, P]
+        L.dsa_index_prefill_pruned.restype = I
         L.dsa_index_decode_noalloc.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P]
         L.dsa_index_decode_noalloc.restype = I
         L.dsa_index_device_status.argtypes = [P, P, P]
@@ -144,6 +148,51 @@ def dsa_index_prefill(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offse
                                        T_k, H, d, int(topk), out_idx.data_ptr(),
                                        out_score.data_ptr(), ws.data_ptr(), ws.numel(),
                                        _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+class _Stats(ctypes.Structure):
+    _fields_ = [("screened_pairs", ctypes.c_int64), ("survivor_pairs", ctypes.c_int64),
+                ("refined_pairs", ctypes.c_int64), ("records", ctypes.c_int64),
+                ("recovered_rows", ctypes.c_int64)]
+
+
+def dsa_index_prefill_pruned_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int,
+                                             n_seed: int) -> int:
+    return int(lib().dsa_index_prefill_pruned_workspace_bytes(T_q, T_k, H, d, topk, n_seed))
+
+
+def dsa_index_prefill_pruned(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offset: int,
+                             topk: int, seed_idx: torch.Tensor, out_idx=None, out_score=None,
+                             workspace=None, stats: bool = False):
+    """Exact Top-k of a causal prefill chunk with DoSA certified pruning.
+
+    Same result as dsa_index_prefill; seed_idx (n_seed,) int32 on the device
+    lists distinct keys visible to every row (0 <= seed < q_offset).  With
+    stats=True the call synchronises and also returns a dict of counters.
+    """
+    dev = k.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k, "k", torch.bfloat16, 2, dev)
+    _need(seed_idx, "seed_idx", torch.int32, 1, dev)
+    T_q, H, d = q.shape
+    T_k = k.shape[0]
+    n_seed = seed_idx.shape[0]
+    if tuple(w.shape) != (T_q, H) or k.shape[1] != d:
+        raise ValueError("shape mismatch between q (T_q,H,d), w (T_q,H) and k (T_k,d)")
+    out_idx, out_score = _outputs(T_q, topk, dev, out_idx, out_score)
+    nbytes = dsa_index_prefill_pruned_workspace_bytes(T_q, T_k, H, d, topk, max(n_seed, 1))
+    ws = _workspace(nbytes, dev, workspace)
+    st = _Stats()
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_pruned(q.data_ptr(), w.data_ptr(), k.data_ptr(), int(q_offset),
+                                              T_q, T_k, H, d, int(topk), seed_idx.data_ptr(), n_seed,
+                                              out_idx.data_ptr(), out_score.data_ptr(),
+                                              ctypes.byref(st) if stats else None, ws.data_ptr(),
+                                              ws.numel(), _stream_ptr(dev)))
+    if stats:
+        return out_idx, out_score, {f: int(getattr(st, f)) for f, _ in _Stats._fields_}
     return out_idx, out_score
 
 

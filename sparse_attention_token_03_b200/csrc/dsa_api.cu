@@ -13,7 +13,9 @@
 #include <string>
 
 #include "../../include/dsa_index.h"
+#include "dsa_dosa.cuh"
 #include "dsa_kernels.cuh"
+#include "dsa_ptx.cuh"
 
 using namespace dsa;
 
@@ -264,6 +266,66 @@ int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const
 }
 
 // ---------------------------------------------------------------------------
+// Workspace of the pruned (DoSA) prefill.
+// ---------------------------------------------------------------------------
+struct PrunedPlan {
+  PrefillPlan seed;    // seed scoring: gathered seed keys, all visible
+  PrefillPlan dense;   // exact dense recovery of flagged rows
+  PrefillPlan screen;  // screening geometry (16 plan rows per query)
+  DecodePlan refine;   // refine: one "sequence" of survivors per row
+  int cap_row;         // survivor ids kept per row
+  int rec_stride;      // seed records per row (topk rounded up to even)
+  int64_t mask_words;
+  size_t off_stats, off_seed_bits, off_k_seed, off_cand, off_seed_rec, off_tau, off_plan_q, off_plan_s,
+      off_knorm, off_bitmask, off_surv_count, off_surv_ids, off_refine_len, off_row_flags, off_init_thr,
+      off_refine, bytes;
+};
+
+int pruned_cap_row(int64_t T_k, int topk) {
+  // survivor lists hold up to a quarter of the keys (rows with more survivors
+  // than that are recomputed by the dense path)
+  const int64_t c = std::max<int64_t>(T_k / 4, 4 * static_cast<int64_t>(topk));
+  return static_cast<int>(std::min<int64_t>(std::min<int64_t>(c, T_k), int64_t(1) << 30));
+}
+
+PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int topk, int n_seed) {
+  PrunedPlan P{};
+  P.seed = plan_prefill(T_q, n_seed, n_seed - 1, H, topk);
+  P.dense = plan_prefill(T_q, T_k, q_offset, H, topk);
+  P.screen = plan_prefill(T_q, T_k, q_offset, kPlanRows, topk);
+  P.refine = plan_decode(static_cast<int>(T_q), topk);
+  P.cap_row = pruned_cap_row(T_k, topk);
+  P.rec_stride = (topk + 1) & ~1;
+  P.mask_words = (T_k + 31) / 32;
+  size_t off = 256;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  P.off_stats = take(8 * sizeof(unsigned long long));
+  P.off_seed_bits = take(static_cast<size_t>(P.mask_words) * 4);
+  P.off_k_seed = take(static_cast<size_t>(n_seed) * kD * 2);
+  // seed scoring and dense recovery run at different times and share one area
+  const size_t sb = P.seed.bytes, db = P.dense.bytes;
+  P.off_cand = take(std::max(sb, db));
+  P.off_seed_rec = take(static_cast<size_t>(T_q) * P.rec_stride * 8);
+  P.off_tau = take(static_cast<size_t>(T_q) * 4);
+  P.off_plan_q = take(static_cast<size_t>(T_q) * kPlanRows * kD * 2);
+  P.off_plan_s = take(static_cast<size_t>(T_q) * kPlanScalars * 4);
+  P.off_knorm = take(static_cast<size_t>(T_k) * 4);
+  P.off_bitmask = take(static_cast<size_t>(T_q) * P.mask_words * 4);
+  P.off_surv_count = take(static_cast<size_t>(T_q) * 4);
+  P.off_surv_ids = take(static_cast<size_t>(T_q) * P.cap_row * 4);
+  P.off_refine_len = take(static_cast<size_t>(T_q) * 4);
+  P.off_row_flags = take(static_cast<size_t>(T_q) * 4);
+  P.off_init_thr = take(static_cast<size_t>(T_q) * 8);
+  P.off_refine = take(P.refine.bytes);
+  P.bytes = off;
+  return P;
+}
+
+// ---------------------------------------------------------------------------
 // Scratch for dsa_index_decode_noalloc.  The array lives in the library's
 // device image, so every GPU on which the library's kernels are loaded holds
 // it (about 28 MB) until the process exits.  Host code must not hand the
@@ -388,6 +450,255 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
   if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
   return decode_run(q, w, k_cache, seq_len, B, t_cap, H, topk, out_idx, out_score,
                     static_cast<uint8_t*>(workspace), P, true, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                             int64_t T_q, int64_t T_k, int H, int d, int topk, const int32_t* seed_idx,
+                             int n_seed, int32_t* out_idx, float* out_score, dsa_stats* stats,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (T_q < 0 || T_k < 1 || q_offset < 0 || q_offset + T_q > T_k)
+    return fail(DSA_EINVAL, "need T_q >= 0, T_k >= 1, 0 <= q_offset, q_offset + T_q <= T_k");
+  if (T_k >= (int64_t(1) << 31) || T_q * H >= (int64_t(1) << 31) || T_q * kPlanRows >= (int64_t(1) << 31))
+    return fail(DSA_EINVAL, "T_k and T_q*H must be below 2^31");
+  if (T_q > 65536) return fail(DSA_EINVAL, "the pruned path takes at most 65536 query rows per call");
+  if (n_seed < topk || n_seed > q_offset)
+    return fail(DSA_ESEED, "need topk <= n_seed <= q_offset (seeds are keys visible to every row), got n_seed = %d",
+                n_seed);
+  if (stats) std::memset(stats, 0, sizeof(dsa_stats));
+  if (T_q == 0) return DSA_OK;
+  if (!q || !w || !k || !seed_idx || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
+      !aligned(seed_idx, 4) || !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
+  const PrunedPlan P = plan_pruned(T_q, T_k, q_offset, H, topk, n_seed);
+  if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  auto at = [&](size_t off) { return ws + off; };
+  cudaError_t e;
+  // zeroed state: status word, counters, seed bitmap, survivor counts
+  if ((e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if ((e = cudaMemsetAsync(at(P.off_stats), 0, 8 * sizeof(unsigned long long), st)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync");
+  if ((e = cudaMemsetAsync(at(P.off_seed_bits), 0, P.mask_words * 4, st)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync");
+  if ((e = cudaMemsetAsync(at(P.off_surv_count), 0, T_q * 4, st)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync");
+  prof_begin(st);
+
+  // 1. seeds: validate, mark, gather
+  SeedPrepParams sp0{seed_idx, n_seed, q_offset, k, reinterpret_cast<uint32_t*>(at(P.off_seed_bits)),
+                     reinterpret_cast<uint16_t*>(at(P.off_k_seed)), err};
+  if ((e = launch_seed_prep(sp0, st)) != cudaSuccess) return cuda_fail(e, "seed prep launch");
+  prof_mark(st, "seed_prep");
+  // 2. seed scores with all heads; per row: sorted seed Top-k records and tau
+  CUtensorMap tq, tk, tks, tplan, tqrow;
+  if ((rc = make_tmap(&tq, q, T_q * H, P.seed.G * H)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tks, at(P.off_k_seed), n_seed, kTileKeys)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tplan, at(P.off_plan_q), T_q * kPlanRows, P.screen.G * kPlanRows)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tqrow, q, T_q * H, H)) != DSA_OK) return rc;
+  {
+    ScoreParams s1{};
+    s1.mode = kModeGathered;
+    s1.topk = topk;
+    s1.lay = P.seed.lay;
+    s1.S = P.seed.S;
+    s1.n_groups = P.seed.n_groups;
+    s1.n_units = P.seed.n_units;
+    s1.q_offset = 0;
+    s1.T_q = T_q;
+    s1.T_k = n_seed;
+    s1.w = w;
+    s1.key_ids = seed_idx;
+    s1.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + P.seed.off_cand));
+    s1.meta = reinterpret_cast<int32_t*>(at(P.off_cand + P.seed.off_meta));
+    s1.err = err;
+    if ((e = launch_score(H, P.seed.G, tq, tks, s1, P.seed.grid, st)) != cudaSuccess)
+      return cuda_fail(e, "seed score launch");
+    prof_mark(st, "seed_score");
+    SelectParams s2{};
+    s2.mode = kModePrefill;
+    s2.G = P.seed.G;
+    s2.S = P.seed.S;
+    s2.topk = topk;
+    s2.lay = P.seed.lay;
+    s2.n_rows = T_q;
+    s2.cand = s1.cand;
+    s2.meta = s1.meta;
+    s2.out_rec = reinterpret_cast<uint64_t*>(at(P.off_seed_rec));
+    s2.rec_stride = P.rec_stride;
+    s2.out_kth = reinterpret_cast<float*>(at(P.off_tau));
+    s2.err = err;
+    if ((e = launch_select(s2, st)) != cudaSuccess) return cuda_fail(e, "seed select launch");
+    prof_mark(st, "seed_select");
+  }
+  // 3. screening plan per row, key norms
+  {
+    PlanParams pp{q, w, reinterpret_cast<const uint16_t*>(at(P.off_k_seed)), n_seed, T_q,
+                  reinterpret_cast<const float*>(at(P.off_tau)), reinterpret_cast<uint16_t*>(at(P.off_plan_q)),
+                  reinterpret_cast<float*>(at(P.off_plan_s))};
+    if ((e = launch_plan(H, pp, st)) != cudaSuccess) return cuda_fail(e, "plan launch");
+    prof_mark(st, "plan");
+    if ((e = launch_keynorm(k, T_k, reinterpret_cast<float*>(at(P.off_knorm)), st)) != cudaSuccess)
+      return cuda_fail(e, "keynorm launch");
+    prof_mark(st, "keynorm");
+  }
+  // 4. screen every visible non-seed key: bound -> survivor bitmask
+  {
+    ScoreParams s3{};
+    s3.mode = kModePrefill;
+    s3.topk = topk;
+    s3.lay = P.screen.lay;
+    s3.S = P.screen.S;
+    s3.n_groups = P.screen.n_groups;
+    s3.n_units = P.screen.n_units;
+    s3.q_offset = q_offset;
+    s3.T_q = T_q;
+    s3.T_k = T_k;
+    s3.err = err;
+    s3.plan_s = reinterpret_cast<const float*>(at(P.off_plan_s));
+    s3.knorm = reinterpret_cast<const float*>(at(P.off_knorm));
+    s3.seed_bits = reinterpret_cast<const uint32_t*>(at(P.off_seed_bits));
+    s3.bitmask = reinterpret_cast<uint32_t*>(at(P.off_bitmask));
+    s3.mask_words = P.mask_words;
+    s3.surv_count = reinterpret_cast<int32_t*>(at(P.off_surv_count));
+    if ((e = launch_screen(tplan, tk, s3, P.screen.grid, st)) != cudaSuccess) return cuda_fail(e, "screen launch");
+    prof_mark(st, "screen");
+  }
+  // 5. compact survivors into id lists; flag rows for recovery
+  CompactParams cp{T_q, q_offset, topk, reinterpret_cast<const uint32_t*>(at(P.off_bitmask)), P.mask_words,
+                   reinterpret_cast<const int32_t*>(at(P.off_surv_count)), P.cap_row,
+                   reinterpret_cast<int32_t*>(at(P.off_surv_ids)), reinterpret_cast<int32_t*>(at(P.off_refine_len)),
+                   reinterpret_cast<int32_t*>(at(P.off_row_flags)), reinterpret_cast<const uint64_t*>(at(P.off_seed_rec)),
+                   P.rec_stride, reinterpret_cast<uint64_t*>(at(P.off_init_thr)), err};
+  if ((e = launch_compact(cp, st)) != cudaSuccess) return cuda_fail(e, "compact launch");
+  prof_mark(st, "compact");
+  // 6. refine survivors exactly (all heads), keeping records at or above the
+  //    row's topk-th seed record, then the final exact Top-k over seed records
+  //    and refined candidates
+  {
+    uint8_t* rws = at(P.off_refine);
+    const DecodePlan& R = P.refine;
+    DecodePlanParams dp{};
+    dp.B = static_cast<int>(T_q);
+    dp.grid = R.grid;
+    dp.t_cap = P.cap_row;
+    dp.seq_len = reinterpret_cast<const int32_t*>(at(P.off_refine_len));
+    dp.seq_start = reinterpret_cast<int64_t*>(rws + R.off_seq_start);
+    dp.unit_tab = reinterpret_cast<int32_t*>(rws + R.off_unit_tab);
+    dp.cta_ubeg = reinterpret_cast<int32_t*>(rws + R.off_cta_ubeg);
+    dp.seq_ubeg = reinterpret_cast<int32_t*>(rws + R.off_seq_ubeg);
+    dp.seq_ucnt = reinterpret_cast<int32_t*>(rws + R.off_seq_ucnt);
+    dp.err = err;
+    if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "refine plan launch");
+    ScoreParams s4{};
+    s4.mode = kModeRefine;
+    s4.topk = topk;
+    s4.lay = R.lay;
+    s4.S = 1;
+    s4.T_k = T_k;
+    s4.w = w;
+    s4.seq_len = dp.seq_len;
+    s4.unit_tab = dp.unit_tab;
+    s4.cta_ubeg = dp.cta_ubeg;
+    s4.cand = reinterpret_cast<uint64_t*>(rws + R.off_cand);
+    s4.meta = reinterpret_cast<int32_t*>(rws + R.off_meta);
+    s4.err = err;
+    s4.surv_ids = reinterpret_cast<const int32_t*>(at(P.off_surv_ids));
+    s4.surv_stride = P.cap_row;
+    s4.k_gather = k;
+    s4.init_thr = reinterpret_cast<const uint64_t*>(at(P.off_init_thr));
+    if ((e = launch_score(H, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
+    prof_mark(st, "refine");
+    SelectParams s5{};
+    s5.mode = kModeDecode;
+    s5.G = 1;
+    s5.S = 1;
+    s5.topk = topk;
+    s5.lay = R.lay;
+    s5.n_rows = T_q;
+    s5.cand = s4.cand;
+    s5.meta = s4.meta;
+    s5.seq_ubeg = dp.seq_ubeg;
+    s5.seq_ucnt = dp.seq_ucnt;
+    s5.extra_rec = reinterpret_cast<const uint64_t*>(at(P.off_seed_rec));
+    s5.rec_stride = P.rec_stride;
+    s5.out_idx = out_idx;
+    s5.out_score = out_score;
+    s5.err = err;
+    if ((e = launch_select(s5, st)) != cudaSuccess) return cuda_fail(e, "final select launch");
+    prof_mark(st, "final_select");
+  }
+  // 7. exact recovery: flagged rows are recomputed by the dense path
+  {
+    ScoreParams s6{};
+    s6.mode = kModePrefill;
+    s6.topk = topk;
+    s6.lay = P.dense.lay;
+    s6.S = P.dense.S;
+    s6.n_groups = P.dense.n_groups;
+    s6.n_units = P.dense.n_units;
+    s6.q_offset = q_offset;
+    s6.T_q = T_q;
+    s6.T_k = T_k;
+    s6.w = w;
+    s6.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + P.dense.off_cand));
+    s6.meta = reinterpret_cast<int32_t*>(at(P.off_cand + P.dense.off_meta));
+    s6.err = err;
+    s6.row_flags = reinterpret_cast<const int32_t*>(at(P.off_row_flags));
+    CUtensorMap tqd;
+    if ((rc = make_tmap(&tqd, q, T_q * H, P.dense.G * H)) != DSA_OK) return rc;
+    if ((e = launch_score(H, P.dense.G, tqd, tk, s6, P.dense.grid, st)) != cudaSuccess)
+      return cuda_fail(e, "recovery launch");
+    SelectParams s7{};
+    s7.mode = kModePrefill;
+    s7.G = P.dense.G;
+    s7.S = P.dense.S;
+    s7.topk = topk;
+    s7.lay = P.dense.lay;
+    s7.n_rows = T_q;
+    s7.cand = s6.cand;
+    s7.meta = s6.meta;
+    s7.out_idx = out_idx;
+    s7.out_score = out_score;
+    s7.row_flags = s6.row_flags;
+    s7.err = err;
+    if ((e = launch_select(s7, st)) != cudaSuccess) return cuda_fail(e, "recovery select launch");
+    prof_mark(st, "recovery");
+  }
+  if (stats) {
+    unsigned long long* cnt = reinterpret_cast<unsigned long long*>(at(P.off_stats));
+    if ((e = launch_stats(reinterpret_cast<const int32_t*>(at(P.off_surv_count)),
+                          reinterpret_cast<const int32_t*>(at(P.off_refine_len)),
+                          reinterpret_cast<const int32_t*>(at(P.off_row_flags)), T_q, cnt, st)) != cudaSuccess)
+      return cuda_fail(e, "stats launch");
+    unsigned long long h[8] = {};
+    uint32_t status = 0;
+    if ((e = cudaMemcpyAsync(h, cnt, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(&status, err, 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      return cuda_fail(e, "reading the pruned-path counters");
+    // screened: every visible key of every row except the row's seeds
+    const int64_t vis = (2 * q_offset + T_q + 1) * T_q / 2;
+    stats->screened_pairs = vis - T_q * static_cast<int64_t>(n_seed);
+    stats->survivor_pairs = static_cast<int64_t>(h[0]);
+    stats->refined_pairs = static_cast<int64_t>(h[1]);
+    stats->recovered_rows = static_cast<int64_t>(h[2]);
+    stats->records = T_q * static_cast<int64_t>(topk) + static_cast<int64_t>(h[1]);
+    if (status & kErrSeed) return fail(DSA_ESEED, "a seed was out of range or repeated; the rows were recomputed densely");
+    if (status & kErrTimeout) return fail(DSA_EDEVICE, "a device-side wait gave up (status 0x%x)", status);
+  }
+  return DSA_OK;
+}
+
+size_t dsa_index_prefill_pruned_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk, int n_seed) {
+  if (check_shape(H, d, topk) != DSA_OK || T_q < 0 || T_k < 1 || n_seed < 1) return 0;
+  return plan_pruned(T_q, T_k, T_k - T_q, H, topk, n_seed).bytes;
 }
 
 int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const uint16_t* k_cache,

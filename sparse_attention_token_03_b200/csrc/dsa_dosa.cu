@@ -1,0 +1,409 @@
+// Support kernels of the DoSA certified-pruning path ("DoSA: Dots Sparse
+// Attention", steps 1-3; 163.com write-up, sections 03-04).
+//
+//   seed_prep_kernel    validate the seed list, mark it in a key bitmap and
+//                       gather the seed keys into a contiguous matrix
+//   keynorm_kernel      ||k_s|| for every key, rounded up
+//   plan_kernel         per query row: retained heads, least-squares residual
+//                       bound, folded positive / negative auxiliary rows and
+//                       the scalars of the screening bound
+//   compact_kernel      survivor bitmask -> ascending survivor id list per row
+//   stats_kernel        counters for the dsa_stats struct
+//
+// The screening MMA and the exact refine are variants of the fused score
+// kernel (dsa_score.cu); the final merge is the shared select kernel.
+#include <cfloat>
+
+#include "dsa_dosa.cuh"
+#include "dsa_ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+// Round an fp32 value to bf16 (nearest, ties to even); finite inputs.
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  uint32_t u = __float_as_uint(f);
+  const uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return static_cast<uint16_t>(u >> 16);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Seeds: every seed must be a distinct key visible to every row of the chunk
+// (0 <= seed < q_offset), so that the topk-th largest seed score is a lower
+// bound on every row's true topk-th score ("DoSA", step 1).
+// ---------------------------------------------------------------------------
+__global__ void seed_prep_kernel(const SeedPrepParams p) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;  // one thread per (seed, 16-byte chunk)
+  const int seed = i >> 4, chunk = i & 15;
+  if (seed >= p.n_seed) return;
+  int32_t id = p.seed_idx[seed];
+  if (id < 0 || id >= p.q_offset) {
+    if (chunk == 0) atomicOr(p.err, kErrSeed);
+    id = 0;  // gather something in bounds; the call recovers densely
+  } else if (chunk == 0) {
+    const uint32_t bit = 1u << (id & 31);
+    const uint32_t old = atomicOr(&p.seed_bits[id >> 5], bit);
+    if (old & bit) atomicOr(p.err, kErrSeed);  // duplicate
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(p.k + static_cast<size_t>(id) * kD);
+  uint4* dst = reinterpret_cast<uint4*>(p.k_seed + static_cast<size_t>(seed) * kD);
+  dst[chunk] = src[chunk];
+}
+
+// ||k_s|| in fp32, rounded up by a relative 2^-12 so that it bounds the exact
+// norm despite the fp32 sum of squares.
+__global__ void keynorm_kernel(const uint16_t* __restrict__ k, int64_t T_k, float* __restrict__ knorm) {
+  const int64_t key = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  const int part = threadIdx.x & 15;  // 16 lanes per key, 8 values each
+  float acc = 0.0f;
+  if (key < T_k) {
+    const uint4 v = reinterpret_cast<const uint4*>(k + key * kD)[part];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      acc = fmaf(lo, lo, acc);
+      acc = fmaf(hi, hi, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (key < T_k && part == 0) knorm[key] = sqrtf(acc) * (1.0f + 1.0f / 4096.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Screening plan of one query row (one CTA of 128 threads per row).
+//
+//  importance_j = |w_j| * sum over sampled seeds s of max(q_j . k_s, 0)
+//  R            = the kRetained heads of largest importance (ties: smaller j)
+//  P / N        = omitted heads with w_j > 0 / w_j < 0
+//  for j in P   c_j = least-squares coefficients of q_j on {q_i, i in R}
+//               (zero if the Gram matrix is not positive definite: any
+//               coefficients keep the bound valid), rho_j = ||q_j - sum c q_i||
+//  alpha_i = sum_P w_j |c_ji|,  beta = sum_P w_j rho_j
+//  q_pos = sum_P w_j q_j, q_neg = sum_N |w_j| q_j (rounded to bf16 for the MMA)
+// With d = q . k, the screening bound (see the screen epilogue) is
+//  U = sum_R [w_i max(d_i,0) + alpha_i |d_i| / 2] + d_pos/2 - max(d_neg,0) + C ||k||
+//  C = beta/2 + ||q_pos - bf16(q_pos)||/2 + ||q_neg - bf16(q_neg)|| + 2^-10 S,
+//  S = sum_j |w_j| ||q_j|| + ||q_pos|| + ||q_neg|| + sum_R alpha_i ||q_i||,
+// where the last term absorbs the fp32 tensor-core accumulation and the fp32
+// arithmetic of the bound and of the exact score (each far below 2^-10 S ||k||).
+// ---------------------------------------------------------------------------
+template <int H>
+__global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
+  constexpr int NT = 128, NSAMP = 64, R = kRetained;
+  __shared__ uint16_t qf[H][kD + 2];  // bf16 bits (padded rows: no bank conflicts)
+  __shared__ uint16_t kf[NSAMP][kD];  // bf16 bits
+  __shared__ float part[NT];
+  __shared__ float imp[H];
+  __shared__ float qn[H];      // ||q_j||
+  __shared__ int sel[R];
+  __shared__ double Lc[R][R];  // Cholesky factor of the retained Gram matrix
+  __shared__ int chol_ok;
+  __shared__ float coef[4][R];  // per-warp least-squares coefficients
+  __shared__ float wal[4][R];   // per-warp alpha partials
+  __shared__ float wbe[4];      // per-warp beta partials
+  __shared__ float red[4];
+
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uint16_t* qrow = p.q + static_cast<size_t>(t) * H * kD;
+  const float* wrow = p.w + static_cast<size_t>(t) * H;
+
+  for (int i = tid; i < H * kD; i += NT) qf[i / kD][i % kD] = qrow[i];
+  const int nsamp = p.n_seed < NSAMP ? p.n_seed : NSAMP;
+  for (int i = tid; i < nsamp * kD; i += NT) {
+    const int s = i / kD;
+    const int pos = static_cast<int>(((2LL * s + 1) * p.n_seed) / (2LL * nsamp));
+    kf[s][i % kD] = p.k_seed[static_cast<size_t>(pos) * kD + (i % kD)];
+  }
+  __syncthreads();
+
+  // importance: NT / H threads per head, each over a fixed slice of samples
+  {
+    constexpr int TPH = NT / H;
+    const int j = tid % H, slice = tid / H;
+    float acc = 0.0f;
+    for (int s = slice; s < nsamp; s += TPH) {
+      float d = 0.0f;
+      for (int e = 0; e < kD; ++e) d = fmaf(bf16_to_f32(qf[j][e]), bf16_to_f32(kf[s][e]), d);
+      acc += fmaxf(d, 0.0f);
+    }
+    part[tid] = acc;
+    __syncthreads();
+    if (tid < H) {
+      float v = 0.0f;
+      for (int sl = 0; sl < TPH; ++sl) v += part[sl * H + tid];
+      imp[tid] = fabsf(wrow[tid]) * v;
+    }
+    // ||q_j||
+    if (tid < H) {
+      float n2 = 0.0f;
+      for (int e = 0; e < kD; ++e) n2 = fmaf(bf16_to_f32(qf[tid][e]), bf16_to_f32(qf[tid][e]), n2);
+      qn[tid] = sqrtf(n2) * (1.0f + 1.0f / 4096.0f);
+    }
+    __syncthreads();
+  }
+  // retained heads: largest importance first, smaller index on ties
+  if (tid == 0) {
+    unsigned long long taken = 0ull;
+    for (int a = 0; a < R; ++a) {
+      int best = -1;
+      for (int j = 0; j < H; ++j) {
+        if ((taken >> j) & 1ull) continue;
+        if (best < 0 || imp[j] > imp[best]) best = j;
+      }
+      sel[a] = best;
+      taken |= 1ull << best;
+    }
+  }
+  __syncthreads();
+  // Gram matrix of the retained rows (fp32 dots, fp64 factorisation)
+  for (int ab = wid; ab < R * R; ab += 4) {
+    const int a = ab / R, b = ab % R;
+    if (b > a) continue;
+    float v = 0.0f;
+    for (int e = lane; e < kD; e += 32) v = fmaf(bf16_to_f32(qf[sel[a]][e]), bf16_to_f32(qf[sel[b]][e]), v);
+    v = warp_sum(v);
+    if (lane == 0) Lc[a][b] = v;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int ok = 1;
+    for (int j = 0; j < R && ok; ++j) {
+      double s = Lc[j][j];
+      for (int k2 = 0; k2 < j; ++k2) s -= Lc[j][k2] * Lc[j][k2];
+      if (!(s > 1e-9 * (1.0 + fabs(Lc[j][j])))) { ok = 0; break; }
+      const double ljj = sqrt(s);
+      Lc[j][j] = ljj;
+      for (int i = j + 1; i < R; ++i) {
+        double v = Lc[i][j];
+        for (int k2 = 0; k2 < j; ++k2) v -= Lc[i][k2] * Lc[j][k2];
+        Lc[i][j] = v / ljj;
+      }
+    }
+    chol_ok = ok;
+  }
+  for (int i = tid; i < 4 * R; i += NT) (&wal[0][0])[i] = 0.0f;
+  if (tid < 4) wbe[tid] = 0.0f;
+  __syncthreads();
+
+  // positive omitted heads: one warp per head, warps take heads in turn
+  for (int j = wid; j < H; j += 4) {
+    bool retained = false;
+    for (int a = 0; a < R; ++a) retained = retained || (sel[a] == j);
+    const float wj = wrow[j];
+    if (retained || !(wj > 0.0f)) continue;
+    float b[R];
+#pragma unroll
+    for (int a = 0; a < R; ++a) {
+      float v = 0.0f;
+      for (int e = lane; e < kD; e += 32) v = fmaf(bf16_to_f32(qf[sel[a]][e]), bf16_to_f32(qf[j][e]), v);
+      b[a] = warp_sum(v);
+    }
+    if (lane == 0) {
+      double x[R];
+      for (int a = 0; a < R; ++a) x[a] = chol_ok ? static_cast<double>(b[a]) : 0.0;
+      if (chol_ok) {
+        for (int i = 0; i < R; ++i) {
+          double v = x[i];
+          for (int k2 = 0; k2 < i; ++k2) v -= Lc[i][k2] * x[k2];
+          x[i] = v / Lc[i][i];
+        }
+        for (int i = R - 1; i >= 0; --i) {
+          double v = x[i];
+          for (int k2 = i + 1; k2 < R; ++k2) v -= Lc[k2][i] * x[k2];
+          x[i] = v / Lc[i][i];
+        }
+      }
+      for (int a = 0; a < R; ++a) coef[wid][a] = static_cast<float>(x[a]);
+    }
+    __syncwarp();
+    float r2 = 0.0f;
+    for (int e = lane; e < kD; e += 32) {
+      float r = bf16_to_f32(qf[j][e]);
+      for (int a = 0; a < R; ++a) r = fmaf(-coef[wid][a], bf16_to_f32(qf[sel[a]][e]), r);
+      r2 = fmaf(r, r, r2);
+    }
+    r2 = warp_sum(r2);
+    if (lane == 0) {
+      const float rho = sqrtf(r2) * (1.0f + 1.0f / 4096.0f);
+      wbe[wid] += wj * rho;
+      for (int a = 0; a < R; ++a) wal[wid][a] += wj * fabsf(coef[wid][a]);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // folded auxiliary rows (thread e owns element e), in ascending head order
+  {
+    const int e = tid;
+    float pos = 0.0f, neg = 0.0f;
+    for (int j = 0; j < H; ++j) {
+      bool retained = false;
+      for (int a = 0; a < R; ++a) retained = retained || (sel[a] == j);
+      if (retained) continue;
+      const float wj = wrow[j];
+      if (wj > 0.0f) pos = fmaf(wj, bf16_to_f32(qf[j][e]), pos);
+      else if (wj < 0.0f) neg = fmaf(-wj, bf16_to_f32(qf[j][e]), neg);
+    }
+    const uint16_t bp = f32_to_bf16(pos), bn = f32_to_bf16(neg);
+    uint16_t* prow = p.plan_q + static_cast<size_t>(t) * kPlanRows * kD;
+    prow[kRetained * kD + e] = bp;
+    prow[(kRetained + 1) * kD + e] = bn;
+    for (int a = 0; a < R; ++a) prow[a * kD + e] = qrow[sel[a] * kD + e];
+    const float dp = pos - bf16_to_f32(bp), dn = neg - bf16_to_f32(bn);
+    // reduce: ||pos||^2, ||neg||^2, ||dp||^2, ||dn||^2
+    float v[4] = {pos * pos, neg * neg, dp * dp, dn * dn};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = warp_sum(v[i]);
+    __shared__ float r4[4][4];
+    if (lane == 0)
+      for (int i = 0; i < 4; ++i) r4[wid][i] = v[i];
+    __syncthreads();
+    if (tid == 0) {
+      float n[4];
+      for (int i = 0; i < 4; ++i) n[i] = sqrtf(((r4[0][i] + r4[1][i]) + r4[2][i]) + r4[3][i]) * (1.0f + 1.0f / 4096.0f);
+      float alpha[R];
+      float beta = ((wbe[0] + wbe[1]) + wbe[2]) + wbe[3];
+      float S = 0.0f;
+      for (int j = 0; j < H; ++j) S += fabsf(wrow[j]) * qn[j];
+      S += n[0] + n[1];
+      for (int a = 0; a < R; ++a) {
+        alpha[a] = ((wal[0][a] + wal[1][a]) + wal[2][a]) + wal[3][a];
+        S += alpha[a] * qn[sel[a]];
+      }
+      float* ps = p.plan_s + static_cast<size_t>(t) * kPlanScalars;
+      for (int a = 0; a < R; ++a) {
+        ps[a] = wrow[sel[a]];
+        ps[kRetained + a] = 0.5f * alpha[a];
+      }
+      const float C = 0.5f * beta + 0.5f * n[2] + n[3] + S * (1.0f / 1024.0f);
+      ps[28] = C * (1.0f + 1.0f / 1024.0f);
+      ps[29] = p.tau[t];
+      ps[30] = 0.0f;
+      ps[31] = 0.0f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Survivor bitmask of one row -> ascending list of survivor key ids (one CTA
+// of 256 threads per row).  Rows whose survivors exceed the list capacity, or
+// all rows when the seed list was invalid, are flagged for the exact dense
+// recovery pass and get an empty refine list.  Also sets the row's refine
+// admission threshold: its topk-th seed record.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
+  __shared__ int s_scan[256 / 32];
+  __shared__ int s_base;
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int count = p.surv_count[t];
+  const bool bad_seed = (*p.err & kErrSeed) != 0;
+  if (tid == 0) p.init_thr[t] = p.seed_rec[static_cast<size_t>(t) * p.rec_stride + p.topk - 1];
+  if (bad_seed || count > p.cap_row) {
+    if (tid == 0) {
+      p.row_flags[t] = 1;
+      p.refine_len[t] = 0;
+    }
+    return;
+  }
+  if (tid == 0) {
+    p.row_flags[t] = 0;
+    p.refine_len[t] = count;
+    s_base = 0;
+  }
+  __syncthreads();
+  const int64_t pos = p.q_offset + t;
+  const int64_t words = pos / 32 + 1;
+  const uint32_t* bm = p.bitmask + static_cast<size_t>(t) * p.mask_words;
+  int32_t* ids = p.surv_ids + static_cast<size_t>(t) * p.cap_row;
+  for (int64_t base = 0; base < words; base += 256) {
+    const int64_t wi = base + tid;
+    uint32_t word = wi < words ? bm[wi] : 0u;
+    if (wi == words - 1 && (pos & 31) != 31) word &= (2u << (pos & 31)) - 1u;  // keys beyond pos
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_scan[wid] = incl;
+    __syncthreads();
+    int before = s_base;
+    for (int w2 = 0; w2 < wid; ++w2) before += s_scan[w2];
+    int at = before + incl - c;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      word &= word - 1;
+      if (at < p.cap_row) ids[at] = static_cast<int32_t>(wi * 32 + b);
+      ++at;
+    }
+    __syncthreads();
+    if (tid == 255) s_base = before + incl;
+    __syncthreads();
+  }
+}
+
+// Sums for dsa_stats (one CTA): survivor pairs, refined pairs, flagged rows.
+__global__ void __launch_bounds__(256) stats_kernel(const int32_t* surv_count, const int32_t* refine_len,
+                                                     const int32_t* row_flags, int64_t T_q,
+                                                     unsigned long long* out) {
+  unsigned long long a = 0, b = 0, c = 0;
+  for (int64_t t = threadIdx.x; t < T_q; t += blockDim.x) {
+    a += static_cast<unsigned long long>(surv_count[t]);
+    b += static_cast<unsigned long long>(refine_len[t]);
+    c += row_flags[t] ? 1ull : 0ull;
+  }
+  atomicAdd(&out[0], a);
+  atomicAdd(&out[1], b);
+  atomicAdd(&out[2], c);
+}
+
+cudaError_t launch_seed_prep(const SeedPrepParams& p, cudaStream_t st) {
+  const int threads = 256;
+  const int64_t n = static_cast<int64_t>(p.n_seed) * 16;
+  seed_prep_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_keynorm(const uint16_t* k, int64_t T_k, float* knorm, cudaStream_t st) {
+  const int threads = 256;
+  const int64_t n = T_k * 16;
+  keynorm_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, st>>>(k, T_k, knorm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan(int H, const PlanParams& p, cudaStream_t st) {
+  if (H == 64) plan_kernel<64><<<static_cast<unsigned>(p.T_q), 128, 0, st>>>(p);
+  else if (H == 32) plan_kernel<32><<<static_cast<unsigned>(p.T_q), 128, 0, st>>>(p);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const CompactParams& p, cudaStream_t st) {
+  compact_kernel<<<static_cast<unsigned>(p.T_q), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats(const int32_t* surv_count, const int32_t* refine_len, const int32_t* row_flags,
+                         int64_t T_q, unsigned long long* out, cudaStream_t st) {
+  stats_kernel<<<1, 256, 0, st>>>(surv_count, refine_len, row_flags, T_q, out);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -55,7 +55,21 @@ enum ScoreMode : int {
   kModePrefill = 0,  // query groups of a causal chunk; keys 0..q_offset+t
   kModeDecode = 1,   // one query per sequence; keys 0..seq_len[b]-1 of its own cache
   kModeGathered = 2, // query groups; keys are a gathered list (all visible), ids remapped
+  kModeRefine = 3,   // one query row per unit (table like decode); keys gathered by id
 };
+
+// Epilogue variants of the fused kernel.
+enum ScoreEpilogue : int {
+  kEpiScore = 0,   // weighted ReLU head sum + streaming Top-k admission
+  kEpiScreen = 1,  // DoSA upper bound from the screening plan + survivor ballot bitmask
+};
+
+// DoSA screening plan: rows per query in the screening MMA and the per-row
+// scalars (floats): [0, 14) retained head weights, [14, 28) half of the
+// retained heads' residual coefficients, [28] key-norm coefficient, [29] tau.
+constexpr int kPlanRows = 16;
+constexpr int kRetained = kPlanRows - 2;
+constexpr int kPlanScalars = 32;
 
 struct ScoreParams {
   int mode;
@@ -76,6 +90,21 @@ struct ScoreParams {
   uint64_t* cand;
   int32_t* meta;
   uint32_t* err;
+  const int32_t* row_flags; // prefill: when set, groups without a flagged row do nothing
+  // refine: survivor key ids per row (stride surv_stride), the key matrix they
+  // index, and an initial admission threshold record per row
+  const int32_t* surv_ids;
+  int64_t surv_stride;
+  const uint16_t* k_gather;
+  const uint64_t* init_thr;
+  // screen: plan scalars [T_q][kPlanScalars], key norms [T_k], seed bitmap,
+  // survivor bitmask [T_q][mask_words] and per-row survivor counts
+  const float* plan_s;
+  const float* knorm;
+  const uint32_t* seed_bits;
+  uint32_t* bitmask;
+  int64_t mask_words;
+  int32_t* surv_count;
 };
 
 struct SelectParams {
@@ -87,11 +116,14 @@ struct SelectParams {
   int64_t n_rows;
   const uint64_t* cand;
   const int32_t* meta;
-  const int32_t* seq_ubeg;  // decode
-  const int32_t* seq_ucnt;  // decode
+  const int32_t* seq_ubeg;  // decode / refine
+  const int32_t* seq_ucnt;  // decode / refine
+  const uint64_t* extra_rec;  // optional [n_rows][rec_stride] extra records (0 = none) merged per row
+  int rec_stride;             // row stride of extra_rec / out_rec (>= topk, even)
+  const int32_t* row_flags;   // optional: only rows with a non-zero flag are written
   int32_t* out_idx;         // [n_rows][topk] (may be null when out_rec is set)
   float* out_score;         // [n_rows][topk]
-  uint64_t* out_rec;        // optional [n_rows][topk] records (sorted, 0-padded)
+  uint64_t* out_rec;        // optional [n_rows][rec_stride] records (sorted, 0-padded)
   float* out_kth;           // optional [n_rows] score of the last selected record
   uint32_t* err;
 };
@@ -121,7 +153,8 @@ struct ScoreSmem {
   __host__ __device__ constexpr uint32_t k_stage() const { return 2u * k_sub(); }
   __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
-  __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + n_cols * 4u; }
+  // head weights (score) or screening-plan scalars (screen): 2 KB at least
+  __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + (n_cols > 512 ? n_cols : 512) * 4u; }
   __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + eg * 2048u * 4u; }
   // per query: base count; per (query, warp quarter): published append count
   __host__ __device__ constexpr uint32_t off_count() const { return off_thr() + 8u * 8u; }
@@ -140,6 +173,8 @@ struct ScoreSmem {
 // Launchers (defined in the .cu files).
 cudaError_t launch_score(int H, int G, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                          const ScoreParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_screen(const CUtensorMap& tmap_plan, const CUtensorMap& tmap_k, const ScoreParams& p,
+                          int grid, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 cudaError_t launch_decode_plan(const DecodePlanParams& p, cudaStream_t stream);
 

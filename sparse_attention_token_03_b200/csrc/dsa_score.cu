@@ -201,13 +201,13 @@ struct Unit {
 template <int G>
 __device__ __forceinline__ Unit unit_geometry(const ScoreParams& p, int u, int H) {
   Unit U;
-  if (p.mode == kModeDecode) {
+  if (p.mode == kModeDecode || p.mode == kModeRefine) {
     const int b = p.unit_tab[3 * u + 0];
     U.slot = u;
     U.row0 = b;
     U.rows = 1;
     U.q_row = static_cast<int64_t>(b) * H;
-    U.k_row = static_cast<int64_t>(b) * p.t_cap;
+    U.k_row = (p.mode == kModeDecode) ? static_cast<int64_t>(b) * p.t_cap : 0;
     U.tile_lo = p.unit_tab[3 * u + 1];
     U.tile_hi = p.unit_tab[3 * u + 2];
     U.vis_base = p.seq_len[b];
@@ -230,23 +230,31 @@ __device__ __forceinline__ Unit unit_geometry(const ScoreParams& p, int u, int H
     const int64_t nt = (nkeys + kTileKeys - 1) / kTileKeys;
     U.tile_lo = s * nt / p.S;
     U.tile_hi = (s + 1) * nt / p.S;
+    if (p.row_flags) {  // recovery pass: skip groups whose rows all came out exact
+      bool any = false;
+      for (int i = 0; i < U.rows; ++i) any = any || (p.row_flags[U.row0 + i] != 0);
+      if (!any) U.tile_hi = U.tile_lo;
+    }
   }
   return U;
 }
 
+__device__ __forceinline__ bool tabled(const ScoreParams& p) {
+  return p.mode == kModeDecode || p.mode == kModeRefine;
+}
 __device__ __forceinline__ int cta_unit_begin(const ScoreParams& p) {
-  return (p.mode == kModeDecode) ? p.cta_ubeg[blockIdx.x] : static_cast<int>(blockIdx.x);
+  return tabled(p) ? p.cta_ubeg[blockIdx.x] : static_cast<int>(blockIdx.x);
 }
 __device__ __forceinline__ int cta_unit_end(const ScoreParams& p) {
-  return (p.mode == kModeDecode) ? p.cta_ubeg[blockIdx.x + 1] : p.n_units;
+  return tabled(p) ? p.cta_ubeg[blockIdx.x + 1] : p.n_units;
 }
 __device__ __forceinline__ int cta_unit_step(const ScoreParams& p) {
-  return (p.mode == kModeDecode) ? 1 : static_cast<int>(gridDim.x);
+  return tabled(p) ? 1 : static_cast<int>(gridDim.x);
 }
 
 }  // namespace
 
-template <int H, int G, int NS, int EG>
+template <int H, int G, int NS, int EG, int EPI>
 __global__ void __launch_bounds__(score_threads(EG), 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
@@ -286,7 +294,8 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_k_full(s), 1);
+      // gathered key tiles are signalled by all 32 producer lanes, TMA tiles by one
+      mbar_init(bar_k_full(s), p.mode == kModeRefine ? 32 : 1);
       mbar_init(bar_k_empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -310,7 +319,66 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   if (warp < score_epi_warp0(EG)) {
    // one setmaxnreg for the whole control warpgroup
    if constexpr (EG == 2) regs_dec<kRegsCtl12>();
-   if (warp == 0) {
+   if (warp == 0 && p.mode == kModeRefine) {
+    // ------------------------------------------------ producer (gathered keys)
+    // Survivor keys are gathered row by row with 16-byte cp.async into the
+    // 128B-swizzled layout the MMA reads.  A stage is signalled LAG tiles
+    // later, once its copies are complete and fenced for the async proxy.
+    constexpr int LAG = NS / 2;
+    uint32_t kt = 0, qi = 0, pending = 0;
+    bool ok = true;
+    auto signal_oldest = [&]() {
+      fence_proxy_async_smem();
+      __syncwarp();
+      mbar_arrive(bar_k_full((kt - pending) % NS));
+      --pending;
+    };
+    auto drain = [&]() {
+      cp_async_wait<0>();
+      while (pending > 0) signal_oldest();
+    };
+    for (int u = u_begin; ok && u < u_end; u += u_step) {
+      const Unit U = unit_geometry<G>(p, u, H);
+      if (U.tile_hi <= U.tile_lo) continue;
+      drain();  // the MMA must see this unit's predecessor complete before the query tile changes
+      if (lane == 0) {
+        ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err);
+        if (ok) {
+          mbar_arrive_expect_tx(bar_q_full, L.q_bytes());
+          tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
+          tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
+        }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++qi;
+      const int32_t* ids = p.surv_ids + U.row0 * p.surv_stride;
+      const int64_t n = U.vis_base;
+      for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
+        const int s = kt % NS;
+        if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err))) break;
+        const uint32_t stage = sK + s * L.k_stage();
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = lane + 32 * jj;
+          const int64_t local = t * kTileKeys + j;
+          const int32_t id = ids[local < n ? local : 0];
+          const uint16_t* src = p.k_gather + static_cast<size_t>(id) * kD;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            cp_async16(stage + (c >> 3) * L.k_sub() + j * 128 + (((c & 7) ^ (j & 7)) << 4), src + c * 8);
+        }
+        cp_async_commit();
+        ++kt;
+        ++pending;
+        if (pending > LAG) {
+          cp_async_wait<LAG>();
+          signal_oldest();
+        }
+      }
+    }
+    drain();
+   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
@@ -391,6 +459,88 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       mbar_wait(bar_q_empty, (nq - 1) & 1, &never, p.err);
     }
    }
+  } else if constexpr (EPI == kEpiScreen) {
+    // ------------------------------------------------------------ screen epilogue
+    // DoSA upper bound per (key, query) from the plan's 16 dot products:
+    //   U = sum_i [w_i max(d_i, 0) + (alpha_i / 2) |d_i|] + d_pos / 2
+    //       - max(d_neg, 0) + C ||k||
+    // (retained heads i < 14, folded positive row d_pos, folded negative row
+    // d_neg; C carries the residual, bf16-rounding and fp32 slack terms).  A
+    // visible non-seed key survives unless U < tau ("DoSA", step 2: prune only
+    // when the bound is strictly below the threshold, keep when unsure).
+    if constexpr (EG == 2) regs_inc<kRegsEpi12>();
+    const int e = (warp - score_epi_warp0(EG)) >> 2;
+    const int bar = 1 + e;
+    const int etid = (threadIdx.x - 32 * score_epi_warp0(EG)) & (kEpiThreads - 1);
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const int q_lo = e * GQ;
+    float* s_pl = s_w;  // [G][kPlanScalars]
+    uint32_t at = 0;
+    bool ok = true;
+    for (int u = u_begin; ok && u < u_end; u += u_step) {
+      const Unit U = unit_geometry<G>(p, u, H);
+      epi_sync(bar);
+      for (int i = etid; i < GQ * kPlanScalars; i += kEpiThreads) {
+        const int qq = q_lo + i / kPlanScalars;
+        s_pl[q_lo * kPlanScalars + i] =
+            (qq < U.rows) ? p.plan_s[(U.row0 + qq) * kPlanScalars + (i % kPlanScalars)] : 0.0f;
+      }
+      epi_sync(bar);
+      int surv[GQ];
+#pragma unroll
+      for (int i = 0; i < GQ; ++i) surv[i] = 0;
+      for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
+        const int a = at & 1;
+        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
+        tc_fence_after();
+        const int64_t key_local = t * kTileKeys + row_in_tile;
+        const bool in_range = key_local < p.T_k;
+        const bool is_seed = in_range && ((p.seed_bits[key_local >> 5] >> lane) & 1u);
+        const float kn = in_range ? p.knorm[key_local] : 0.0f;
+        const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                              static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
+        uint32_t xb[2][16];
+        tmem_ld16(trow, xb[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          if (i + 1 < GQ) tmem_ld16(trow + (i + 1) * H, xb[(i + 1) & 1]);
+          const float* pl = s_pl + (q_lo + i) * kPlanScalars;
+          const uint32_t* d = xb[i & 1];
+          float ub = 0.0f;
+#pragma unroll
+          for (int r = 0; r < kRetained; ++r) {
+            const float x = __uint_as_float(d[r]);
+            ub = fmaf(pl[r], fmaxf(x, 0.0f), ub);
+            ub = fmaf(pl[kRetained + r], fabsf(x), ub);
+          }
+          ub = fmaf(0.5f, __uint_as_float(d[kRetained]), ub);
+          ub -= fmaxf(__uint_as_float(d[kRetained + 1]), 0.0f);
+          ub = fmaf(pl[28], kn, ub);
+          const int qq = q_lo + i;
+          const bool vis = qq < U.rows && key_local < U.vis_base + qq && !is_seed;
+          const bool keep = vis && !(ub < pl[29]);
+          const uint32_t word = __ballot_sync(0xFFFFFFFFu, keep);
+          if (lane == 0 && qq < U.rows && (key_local >> 5) < p.mask_words)
+            p.bitmask[(U.row0 + qq) * p.mask_words + (key_local >> 5)] = word;
+          surv[i] += __popc(word);
+          if (i + 1 < GQ) tmem_wait_ld();
+          if (i + 2 == GQ || GQ == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_acc_empty(a));
+          }
+        }
+        ++at;
+      }
+      if (!ok) break;
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < GQ; ++i)
+          if (q_lo + i < U.rows && surv[i] > 0) atomicAdd(&p.surv_count[U.row0 + q_lo + i], surv[i]);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     if constexpr (EG == 2) regs_inc<kRegsEpi12>();
@@ -414,7 +564,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       if (etid < GQ) {
         const int qq = q_lo + etid;
         s_count[qq] = 0;
-        s_thr[qq] = 0ull;
+        s_thr[qq] = (p.init_thr && qq < U.rows) ? p.init_thr[U.row0 + qq] : 0ull;
         s_half[qq] = 0;
 #pragma unroll
         for (int r = 0; r < 4; ++r) s_wcnt[qq * 4 + r] = 0;
@@ -454,6 +604,8 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         const int64_t key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
+        if (p.mode == kModeRefine && key_local < U.vis_base)
+          key_id = static_cast<uint32_t>(p.surv_ids[U.row0 * p.surv_stride + key_local]);
         uint64_t thr[GQ];
         int half[GQ];
 #pragma unroll
@@ -572,12 +724,12 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
-template <int H, int G, int NS, int EG>
+template <int H, int G, int NS, int EG, int EPI = kEpiScore>
 static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const ScoreParams& p, int grid, cudaStream_t stream) {
   constexpr ScoreSmem L{G * H, NS, EG};
   static_assert(L.request() <= 227u * 1024u, "shared memory budget");
-  auto kern = score_topk_kernel<H, G, NS, EG>;
+  auto kern = score_topk_kernel<H, G, NS, EG, EPI>;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool configured[64] = {};
@@ -606,6 +758,12 @@ cudaError_t launch_score(int H, int G, const CUtensorMap& tq, const CUtensorMap&
   if (H == 64 && G == 1) return launch_score_t<64, 1, 6, 1>(tq, tk, p, grid, stream);
   if (H == 32 && G == 1) return launch_score_t<32, 1, 6, 1>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;
+}
+
+// Screening: 16 plan rows per query, 16 queries per MMA (N = 256).
+cudaError_t launch_screen(const CUtensorMap& tplan, const CUtensorMap& tk, const ScoreParams& p,
+                          int grid, cudaStream_t stream) {
+  return launch_score_t<kPlanRows, 16, 4, 2, kEpiScreen>(tplan, tk, p, grid, stream);
 }
 
 }  // namespace dsa

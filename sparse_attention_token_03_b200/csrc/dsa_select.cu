@@ -157,12 +157,18 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
 
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
+  if (p.row_flags && p.row_flags[row] == 0) return;  // row already exact
   const RowUnits R = row_units(p, row);
   const int G = (p.mode == kModeDecode) ? 1 : p.G;
   const CandLayout lay = p.lay;
 
-  // segment sg = 5 * unit + region of the row's candidate buffers
+  // segment sg = 5 * unit + region of the row's candidate buffers; one more
+  // segment holds the row's extra records when given
   auto segment = [&](int sg, int& cnt) -> const uint64_t* {
+    if (sg == 5 * R.n_u) {
+      cnt = p.topk;
+      return p.extra_rec + static_cast<size_t>(row) * p.rec_stride;
+    }
     const int u = sg / 5, r = sg % 5;
     const size_t qi = static_cast<size_t>(R.slot_lo + u) * G + R.q;
     const int32_t* mt = p.meta + qi * kMetaInts;
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     return p.cand + qi * lay.query_recs() + static_cast<size_t>(mt[0] & 1) * lay.half_recs() +
            lay.region_off(r);
   };
-  const int n_seg = 5 * R.n_u;
+  const int n_seg = 5 * R.n_u + (p.extra_rec ? 1 : 0);
 
   if (tid == 0) {
     int n = 0, staged = 0;
@@ -335,6 +341,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   __syncthreads();
   sort2048_desc(v, s_win);
   const size_t o = static_cast<size_t>(row) * p.topk;
+  const size_t orec = static_cast<size_t>(row) * p.rec_stride;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int i = 8 * tid + s;
@@ -342,7 +349,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       const bool ok = i < m;
       if (p.out_idx) p.out_idx[o + i] = ok ? static_cast<int32_t>(record_key(v[s])) : -1;
       if (p.out_score) p.out_score[o + i] = ok ? record_score(v[s]) : -INFINITY;
-      if (p.out_rec) p.out_rec[o + i] = ok ? v[s] : 0ull;
+      if (p.out_rec) p.out_rec[orec + i] = ok ? v[s] : 0ull;
     }
   }
   if (p.out_kth) {

@@ -16,6 +16,13 @@ activations, which are not available here):
   of rank 8 / 16 / 32; queries from the last third's basis; w has magnitude
   |N(0, 1/8)| and is negative with probability 0.4.
 
+``head_rank`` > 0 (any key recipe): a row's H query heads are no longer
+independent draws; they are mixtures of ``head_rank`` per-row latent vectors,
+q_{t,j} = sum_m A_{j,m} b_{t,m} + 0.05 e_{t,j}, with one mixing matrix
+A ~ N(0, 1/head_rank) (H x head_rank) for the whole input and b_{t,m}
+drawn like a query row of the key recipe.  It stands in for index heads that
+are projections of one shared query latent.
+
 Nothing here computes an index score or selects keys.
 """
 
@@ -48,6 +55,7 @@ class Workload:
     rank: int = 16
     n_seed: int = 0  # DoSA seed-set size (0: no seed set)
     n_anchor: int = 0  # seeds taken from an anchor query's selection
+    head_rank: int = 0  # > 0: heads are mixtures of head_rank latent rows
     notes: str = field(default="", compare=False)
 
     @property
@@ -146,9 +154,23 @@ def _weights(rng: np.random.Generator, shape, recipe: str) -> np.ndarray:
     return (rng.standard_normal(shape) * sd).astype(np.float32)
 
 
+def _mix_heads(rng: np.random.Generator, latent: np.ndarray, A: np.ndarray,
+               out: np.ndarray) -> None:
+    """out (rows*H, d) <- bf16 of per-row mixtures A @ latent of the latent rows (rows*r, d)."""
+    H, r = A.shape
+    d = latent.shape[1]
+    rows = latent.shape[0] // r
+    lat = bf16_bits_to_f32(latent).astype(np.float64).reshape(rows, r, d)
+    for s in range(0, rows, 4096):
+        e = min(rows, s + 4096)
+        mix = np.einsum("hm,tmd->thd", A, lat[s:e])
+        noise = 0.05 * rng.standard_normal(mix.shape)
+        out[s * H:e * H] = bf16_bits_from_f64(mix + noise).reshape(-1, d)
+
+
 def make_prefill(wl: Workload | str, *, T_q: int | None = None, T_k: int | None = None,
                  q_offset: int | None = None, seed: int | None = None,
-                 with_anchor: bool = False) -> dict:
+                 with_anchor: bool = False, head_rank: int | None = None) -> dict:
     """Generate q (T_q,H,d) bf16 bits, w (T_q,H) fp32 and k (T_k,d) bf16 bits.
 
     The size overrides make smaller cases of the same recipe.  With
@@ -198,6 +220,25 @@ def make_prefill(wl: Workload | str, *, T_q: int | None = None, T_k: int | None 
             out.update(q_anchor=qa, w_anchor=_weights(rng, (H,), "domains"))
     else:
         raise ValueError(f"unknown key recipe {wl.keys!r}")
+    hr = wl.head_rank if head_rank is None else head_rank
+    if hr > 0:
+        # replace the query heads by mixtures of hr latent rows per query row
+        lat = np.empty((T_q * hr, d), np.uint16)
+        if wl.keys == "gauss":
+            _gauss_rows(rng, T_q * hr, d, 1.0 / np.sqrt(128.0), lat)
+        else:
+            _lowrank_rows(rng, U if wl.keys == "lowrank" else bases[2], T_q * hr, 0.3, lat)
+        A = rng.standard_normal((H, hr)) / np.sqrt(hr)
+        _mix_heads(rng, lat, A, q)
+        if with_anchor:
+            la = np.empty((hr, d), np.uint16)
+            if wl.keys == "gauss":
+                _gauss_rows(rng, hr, d, 1.0 / np.sqrt(128.0), la)
+            else:
+                _lowrank_rows(rng, U if wl.keys == "lowrank" else bases[2], hr, 0.3, la)
+            qa = np.empty((H, d), np.uint16)
+            _mix_heads(rng, la, A, qa)
+            out["q_anchor"] = qa
     out.update(q=q.reshape(T_q, H, d), w=w, k=k, q_offset=q_offset, T_q=T_q, T_k=T_k,
                H=H, d=d, topk=wl.topk)
     return out

@@ -1,0 +1,164 @@
+"""DoSA certified pruning (dsa_index_prefill_pruned) on the GPU.
+
+Its losslessness invariant: on the same inputs the pruned path returns the
+dense path's output bit for bit ("DoSA", the pruned selection keeps the
+original Top-k).  Both are also checked against the fp64 oracle, and the
+recovery paths (bad seeds, survivor overflow) must stay exact.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_token_03_b200 as dsa
+from synth import WORKLOADS, make_prefill, random_distinct_keys
+from tests.parity import check_rows, oracle_prefill_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_inputs(x):
+    return bf16(x["q"]), torch.from_numpy(x["w"]).cuda(), bf16(x["k"])
+
+
+def anchor_seeds(x, topk, n_random, seed):
+    """The recipe of the long-context chunks: the oracle's Top-topk of the
+    query just before the chunk, plus distinct random keys before the chunk."""
+    off = x["q_offset"]
+    qa, wa = x["q_anchor"], x["w_anchor"]
+    idx, _, _ = oracle.prefill_topk(qa[None], wa[None], x["k"][:off], off - 1, topk)
+    anchor = idx[0][idx[0] >= 0]
+    rnd = random_distinct_keys(seed, 0, off, n_random, exclude=anchor)
+    return np.concatenate([anchor, rnd]).astype(np.int32)
+
+
+def run_both(x, topk, seeds):
+    q, w, k = dev_inputs(x)
+    di, ds = dsa.dsa_index_prefill(q, w, k, x["q_offset"], topk)
+    pi, ps, st = dsa.dsa_index_prefill_pruned(q, w, k, x["q_offset"], topk,
+                                              torch.from_numpy(seeds).cuda(), stats=True)
+    torch.cuda.synchronize()
+    return di.cpu().numpy(), ds.cpu().numpy(), pi.cpu().numpy(), ps.cpu().numpy(), st
+
+
+@pytest.mark.parametrize("recipe,H", [("causal_1k_h64", 64), ("causal_16k_h64", 64),
+                                      ("chunk_128k_h32", 32), ("chunk_1m_h64", 64)])
+def test_pruned_equals_dense_bitwise_and_oracle(recipe, H):
+    T_k, off, topk = 1536, 1024, 128
+    x = make_prefill(recipe, T_q=T_k - off, T_k=T_k, q_offset=off, seed=404, with_anchor=True)
+    seeds = anchor_seeds(x, topk, 200, seed=7)
+    di, ds, pi, ps, st = run_both(x, topk, seeds)
+    assert np.array_equal(pi, di), "pruned indices differ from the dense path"
+    assert np.array_equal(ps.view(np.uint32), ds.view(np.uint32)), "pruned scores differ bitwise"
+    rows = np.arange(0, T_k - off, 7)
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
+    check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, f"pruned {recipe}")
+    T_q = T_k - off
+    vis = (2 * off + T_q + 1) * T_q // 2
+    assert st["screened_pairs"] == vis - T_q * len(seeds)
+    assert 0 <= st["survivor_pairs"] <= st["screened_pairs"]
+    assert st["refined_pairs"] <= st["survivor_pairs"]
+    print(recipe, st)
+
+
+@pytest.mark.parametrize("H", [64, 32])
+def test_pruned_refine_path_with_a_tight_bound(H):
+    # Heads built so that the bound is exact up to its safety slack: 14
+    # distinct heads with large weights (the planner retains them) and H-14
+    # identical copies of one vector with small negative weights (no positive
+    # omitted head; folding identical negative heads loses nothing).  The 24
+    # rows repeat one query and the seeds hold its Top-k among the keys before
+    # the chunk, so tau is close to every row's k-th score: nearly every
+    # non-Top-k key is pruned and the result comes from screen -> compact ->
+    # refine, with no dense recovery.
+    T_q, off, topk = 24, 6000, 128
+    x = make_prefill("causal_1k_h64" if H == 64 else "chunk_128k_h32", T_q=T_q, T_k=off + T_q,
+                     q_offset=off, seed=407)
+    rng = np.random.default_rng(0)
+    q0 = x["q"][0].copy()
+    q0[14:] = q0[14]
+    w0 = np.empty(H, np.float32)
+    w0[:14] = rng.standard_normal(14).astype(np.float32) * 4.0
+    w0[14:] = -0.01
+    x["q"][:] = q0
+    x["w"][:] = w0
+    idx, _, _ = oracle.prefill_topk(x["q"][:1], x["w"][:1], x["k"][:off], off - 1, topk)
+    seeds = np.concatenate([idx[0], random_distinct_keys(13, 0, off, 300, exclude=idx[0])]).astype(np.int32)
+    di, ds, pi, ps, st = run_both(x, topk, seeds)
+    print("tight bound", H, st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    assert st["recovered_rows"] == 0
+    assert st["refined_pairs"] == st["survivor_pairs"] > 0
+    assert st["survivor_pairs"] < 0.2 * st["screened_pairs"]
+    rows = np.array([0, 11, 23])
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
+    check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, f"tight {H}")
+
+
+def test_pruned_filter_rate_on_shared_latent_heads():
+    # statistics only (the filter rate depends on the data): heads mixed from
+    # one latent row per query, rows repeating one query
+    T_q, off, topk = 24, 6000, 128
+    x = make_prefill("chunk_1m_h64", T_q=T_q, T_k=off + T_q, q_offset=off, seed=406, head_rank=1)
+    x["q"][1:] = x["q"][0]
+    x["w"][1:] = x["w"][0]
+    idx, _, _ = oracle.prefill_topk(x["q"][:1], x["w"][:1], x["k"][:off], off - 1, topk)
+    seeds = np.concatenate([idx[0], random_distinct_keys(13, 0, off, 300, exclude=idx[0])]).astype(np.int32)
+    di, ds, pi, ps, st = run_both(x, topk, seeds)
+    print("shared latent", st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+
+
+def test_pruned_ragged_chunk_and_small_topk():
+    # a chunk whose rows are not a multiple of any tile or group size
+    x = make_prefill("causal_16k_h64", T_q=37, T_k=3037, q_offset=3000, seed=5, with_anchor=True)
+    seeds = anchor_seeds(x, 9, 300, seed=8)
+    di, ds, pi, ps, st = run_both(x, 9, seeds)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+
+
+def test_pruned_overflowing_rows_are_recovered_exactly():
+    # only topk random seeds: tau is weak, survivors exceed the per-row list
+    # (max(T_k/4, 4 topk) = 2048 keys), and those rows take the dense path
+    x = make_prefill("causal_1k_h64", T_q=40, T_k=8232, q_offset=8192, seed=9)
+    seeds = random_distinct_keys(3, 0, 8192, 64)
+    di, ds, pi, ps, st = run_both(x, 64, seeds)
+    assert st["recovered_rows"] > 0
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+
+
+def test_pruned_bad_seed_lists():
+    x = make_prefill("causal_1k_h64", T_q=16, T_k=600, q_offset=584, seed=10)
+    q, w, k = dev_inputs(x)
+    di, ds = dsa.dsa_index_prefill(q, w, k, 584, 32)
+    # fewer seeds than topk: refused before any launch
+    with pytest.raises(dsa.DSAError, match="ESEED"):
+        dsa.dsa_index_prefill_pruned(q, w, k, 584, 32, torch.arange(31, dtype=torch.int32, device="cuda"))
+    # a repeated seed and a seed that is not visible to every row: detected on
+    # the device, every row recomputed densely, reported with stats
+    for bad in ([5] + list(range(40, 80)) + [5], list(range(0, 40)) + [590]):
+        s = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        with pytest.raises(dsa.DSAError, match="ESEED"):
+            dsa.dsa_index_prefill_pruned(q, w, k, 584, 32, s, stats=True)
+        pi, ps = dsa.dsa_index_prefill_pruned(q, w, k, 584, 32, s)
+        torch.cuda.synchronize()
+        assert torch.equal(pi, di) and torch.equal(ps, ds)
+
+
+@pytest.mark.parametrize("name,n_rows", [("chunk_128k_h32", 6), ("chunk_1m_h64", 4)])
+def test_full_size_pruned_equals_dense(name, n_rows):
+    wl = WORKLOADS[name]
+    x = make_prefill(wl, with_anchor=True)
+    seeds = anchor_seeds(x, wl.topk, wl.n_seed - wl.n_anchor, seed=11)
+    assert len(seeds) == wl.n_seed
+    di, ds, pi, ps, st = run_both(x, wl.topk, seeds)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    rows = np.unique(np.linspace(0, wl.T_q - 1, n_rows).round().astype(np.int64))
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, wl.topk)
+    check_rows(pi[rows], ps[rows], oi, osc, amax, wl.q_offset + rows + 1, wl.topk, score_of, name)
+    print(name, st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
