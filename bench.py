@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--path", choices=["dense", "pruned"], default="dense",
+                    help="prefill path: dense fused scoring, or DoSA certified pruning")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -241,8 +243,11 @@ def main():
     torch.cuda.set_device(dev)
 
     seed = wl.seed + 7919 * rank
+    pruned = args.path == "pruned"
+    if pruned and (wl.kind != "prefill" or wl.n_seed == 0):
+        raise SystemExit(f"--path pruned needs a chunked prefill workload with a seed set, not {wl.name}")
     if wl.kind == "prefill":
-        x = make_prefill(wl, seed=seed)
+        x = make_prefill(wl, seed=seed, with_anchor=pruned)
     else:
         x = make_decode(wl, seed=seed)
 
@@ -254,7 +259,32 @@ def main():
     rows = wl.T_q if wl.kind == "prefill" else wl.B
     out_idx = torch.empty((rows, wl.topk), dtype=torch.int32, device=dev)
     out_score = torch.empty((rows, wl.topk), dtype=torch.float32, device=dev)
-    if wl.kind == "prefill":
+    filter_stats = None
+    if wl.kind == "prefill" and pruned:
+        # seed set: the anchor query's Top-k (the query just before the chunk,
+        # selected by this library's own decode call) plus random keys
+        qa = to_dev_bf16(x["q_anchor"][None])
+        wa = torch.from_numpy(x["w_anchor"][None]).to(dev)
+        ka = k[:wl.q_offset].unsqueeze(0)
+        la = torch.tensor([wl.q_offset], dtype=torch.int32, device=dev)
+        aidx, _ = dsa.dsa_index_decode(qa, wa, ka.contiguous(), la, wl.n_anchor)
+        anchor = aidx[0].cpu().numpy()
+        from synth import random_distinct_keys
+        rnd = random_distinct_keys(seed + 1, 0, wl.q_offset, wl.n_seed - wl.n_anchor, exclude=anchor)
+        seeds = torch.from_numpy(np.concatenate([anchor, rnd]).astype(np.int32)).to(dev)
+        del ka
+        ws = torch.empty(dsa.dsa_index_prefill_pruned_workspace_bytes(wl.T_q, wl.T_k, wl.H, wl.d, wl.topk,
+                                                                      wl.n_seed),
+                         dtype=torch.uint8, device=dev)
+        _, _, filter_stats = dsa.dsa_index_prefill_pruned(q, w, k, wl.q_offset, wl.topk, seeds,
+                                                          out_idx=out_idx, out_score=out_score,
+                                                          workspace=ws, stats=True)
+
+        def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score):
+            dsa.dsa_index_prefill_pruned(qq, ww, kk, wl.q_offset, wl.topk, seeds, out_idx=oi,
+                                         out_score=osc, workspace=ws)
+        n_kernels = 12
+    elif wl.kind == "prefill":
         ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(wl.T_q, wl.T_k, wl.H, wl.d, wl.topk),
                          dtype=torch.uint8, device=dev)
 
@@ -318,7 +348,18 @@ def main():
     # ---- roofline of the dominant kernel (the fused score + Top-k kernel)
     pk, pk_src = peaks()
     score_ms = float(np.mean(kern_ms.get("score_topk", [float("nan")])))
-    if wl.kind == "prefill":
+    if pruned:
+        # the screening MMA dominates: 16 plan rows per query, 2*16*d flops per
+        # visible pair (executed flops, not the dense-equivalent ones)
+        score_ms = float(np.mean(kern_ms.get("screen", [float("nan")])))
+        flops = 2.0 * 16 * wl.d * pairs
+        achieved = flops / (score_ms * 1e-3) / 1e12
+        peak = float(pk["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"bf16_tflops (burst) of {pk_src}",
+                "kernel": "score_topk_kernel (screen variant)", "kernel_ms": score_ms,
+                "traffic": recorded_traffic(wl.name, "screen")}
+    elif wl.kind == "prefill":
         flops = 2.0 * wl.H * wl.d * pairs
         achieved = flops / (score_ms * 1e-3) / 1e12
         peak = float(pk["bf16_tflops"])
@@ -330,9 +371,10 @@ def main():
         peak = float(pk["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"hbm_gbs of {pk_src}"}
-    roof["kernel"] = "score_topk_kernel"
-    roof["kernel_ms"] = score_ms
-    roof["traffic"] = recorded_traffic(wl.name, "score_topk_kernel")
+    if not pruned:
+        roof["kernel"] = "score_topk_kernel"
+        roof["kernel_ms"] = score_ms
+        roof["traffic"] = recorded_traffic(wl.name, "score_topk_kernel")
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -360,6 +402,8 @@ def main():
             if wl.kind == "decode":
                 dsl.copy_(extra["sl"], non_blocking=True)
                 step(dq, dw, dk, out_idx, out_score, dsl)
+            elif pruned:
+                step(dq, dw, dk, out_idx, out_score)
             else:
                 step(dq, dw, dk, out_idx, out_score)
             hoi.copy_(out_idx, non_blocking=True)
@@ -386,15 +430,19 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": "indexer causal q.k pairs/s", "value": value, "unit": "pairs/s",
+            "metric": "indexer causal q.k pairs/s" + (" (effective, DoSA)" if pruned else ""),
+            "value": value, "unit": "pairs/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
-                                                 parallelism=f"replicas x{world}"),
+                                                 parallelism=f"replicas x{world}", path=args.path),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": n_kernels * args.steps, "clocks": clocks, "device_status": status,
             "kernel_ms": {n: float(np.mean(v)) for n, v in kern_ms.items()},
         }
+        if filter_stats is not None:
+            line["dosa"] = dict(filter_stats, filter_rate=1.0 - filter_stats["survivor_pairs"]
+                                / max(filter_stats["screened_pairs"], 1))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
