@@ -37,12 +37,9 @@ namespace {
 // Each epilogue warpgroup e synchronises on named barrier 1 + e.
 __device__ __forceinline__ void epi_sync(int bar) { named_bar_sync(bar, kEpiThreads); }
 
-// Warp-aggregated shared-memory histogram increment.
+// Shared-memory histogram increment.
 __device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t digit) {
-  const uint32_t key = valid ? digit : 0xFFFFFFFFu;
-  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-  const int lane = threadIdx.x & 31;
-  if (valid && lane == (__ffs(peers) - 1)) atomicAdd(&hist[digit], __popc(peers));
+  if (valid) atomicAdd(&hist[digit], 1u);
 }
 
 // Find the digit bucket B holding the need-th largest record:

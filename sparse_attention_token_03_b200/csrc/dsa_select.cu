@@ -24,9 +24,7 @@ namespace {
 constexpr int kStageRecs = 7680;  // candidates of a row staged in shared memory (60 KB)
 
 __device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_t digit) {
-  const uint32_t key = valid ? digit : 0xFFFFFFFFu;
-  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-  if (valid && (threadIdx.x & 31) == (__ffs(peers) - 1)) atomicAdd(&hist[digit], __popc(peers));
+  if (valid) atomicAdd(&hist[digit], 1u);
 }
 
 // Block-wide: largest bucket B with above + sum_{d >= B} hist[d] >= need.
