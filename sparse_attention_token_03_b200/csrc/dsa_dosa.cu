@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
   __shared__ float coef[4][R];  // per-warp least-squares coefficients
   __shared__ float wal[4][R];   // per-warp alpha partials
   __shared__ float wbe[4];      // per-warp beta partials
-  __shared__ float red[4];
 
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;

@@ -33,6 +33,13 @@ static_assert(128 * kRegsCtl12 + 256 * kRegsEpi12 == 384 * kRegsLaunch12, "regis
 constexpr int kSelectThreads = 256;
 
 constexpr int kMetaInts = 8;
+// Score-code histogram of a query's buffered records: bin = code >> 22
+// (sign, exponent and one mantissa bit of the fp32 score: half-octave bins).
+constexpr int kHistBins = 1024;
+constexpr int kHistShift = 22;
+// The epilogue publishes append counts and checks for overflow every
+// kCheckTiles tiles; a warp appends at most 32 records per query per tile.
+constexpr int kCheckTiles = 8;
 
 struct CandLayout {
   int keep_cap;  // records kept by a compaction (>= topk), multiple of 32
@@ -44,9 +51,10 @@ struct CandLayout {
 
 __host__ __device__ constexpr CandLayout cand_layout(int topk) {
   CandLayout L{0, 0};
-  L.keep_cap = ((topk + topk / 2 + 31) / 32) * 32;
-  L.app_cap = (((topk / 2 + 160) + 31) / 32) * 32;  // room for 4 tiles past the check threshold
-  if (L.app_cap < 256) L.app_cap = 256;
+  L.keep_cap = ((2 * topk + 31) / 32) * 32;
+  // a warp's region takes a quarter of topk plus kCheckTiles tiles of appends
+  // past the overflow check
+  L.app_cap = (((topk / 4 + 64 * kCheckTiles) + 31) / 32) * 32;
   return L;
 }
 
@@ -146,19 +154,22 @@ struct DecodePlanParams {
 struct ScoreSmem {
   int n_cols;
   int ns;
-  int eg;  // epilogue warpgroups (each has its own histogram and scratch)
+  int eg;   // epilogue warpgroups
+  int nqh;  // per-query score-code histograms (kHistBins bins each); 0 for the screen
   __host__ __device__ constexpr uint32_t q_sub() const { return static_cast<uint32_t>(n_cols) * 128u; }
   __host__ __device__ constexpr uint32_t q_bytes() const { return 2u * q_sub(); }
   __host__ __device__ constexpr uint32_t k_sub() const { return 128u * 128u; }
   __host__ __device__ constexpr uint32_t k_stage() const { return 2u * k_sub(); }
   __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
-  // head weights (score) or screening-plan scalars (screen): 2 KB at least
-  __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + (n_cols > 512 ? n_cols : 512) * 4u; }
-  __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + eg * 2048u * 4u; }
-  // per query: base count; per (query, warp quarter): published append count
+  // screening-plan scalars (screen): 2 KB
+  __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + 512u * 4u; }
+  __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + nqh * kHistBins * 4u; }
+  // per query: base count, count at the last threshold update; per (query,
+  // warp quarter): published append count
   __host__ __device__ constexpr uint32_t off_count() const { return off_thr() + 8u * 8u; }
-  __host__ __device__ constexpr uint32_t off_wcnt() const { return off_count() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_upd() const { return off_count() + 8u * 4u; }
+  __host__ __device__ constexpr uint32_t off_wcnt() const { return off_upd() + 8u * 4u; }
   __host__ __device__ constexpr uint32_t off_half() const { return off_wcnt() + 32u * 4u; }
   __host__ __device__ constexpr uint32_t off_misc() const { return off_half() + 8u * 4u; }
   __host__ __device__ constexpr uint32_t off_bars() const { return off_misc() + eg * 32u * 4u; }

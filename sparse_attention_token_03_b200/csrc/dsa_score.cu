@@ -48,10 +48,11 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t di
 // tid in [0, 128); nb in {512, 2048}; scratch >= 4 ints.
 __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int need, int tid,
                                 int* scratch, int* res, int bar) {
-  const int bpt = nb / kEpiThreads;
+  const int bpt = (nb + kEpiThreads - 1) / kEpiThreads;
   const int lo = tid * bpt;
   int local = 0;
-  for (int b = 0; b < bpt; ++b) local += hist[lo + b];
+  for (int b = 0; b < bpt; ++b)
+    if (lo + b < nb) local += hist[lo + b];
   // exclusive suffix sum over threads (higher tid = higher digits)
   const int lane = tid & 31, wid = tid >> 5;
   int incl = local;
@@ -68,6 +69,7 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
   if (above + excl < need && above + excl + local >= need) {
     int acc = above + excl;
     for (int b = bpt - 1; b >= 0; --b) {
+      if (lo + b >= nb) continue;
       const int h = hist[lo + b];
       if (acc + h >= need) {
         res[0] = lo + b;
@@ -81,8 +83,8 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
   epi_sync(bar);
 }
 
-// Compact the candidate buffer of one (slot, query), run by its epilogue
-// warpgroup.  The records of the active half (base region + four append
+// Exact fallback compaction of one (slot, query), run by its epilogue
+// warpgroup when the histogram threshold would keep too many records.  The records of the active half (base region + four append
 // regions) are reduced to a superset of the `need` largest ones holding at
 // most lay.keep_cap records, written to the base region of the other half.
 // Radix digits start at the highest bit in which the smallest and largest
@@ -108,7 +110,7 @@ __device__ uint64_t epi_compact(uint64_t* qbuf, const CandLayout lay, int q, int
   }
   uint64_t thr = lo;
   for (int pass = 0; pass < 7 && diff != 0; ++pass) {
-    const int shift = max(64 - pbits - 11, 0);
+    const int shift = max(64 - pbits - 10, 0);
     const int width = 64 - pbits - shift;
     const int nb = 1 << width;
     for (int i = tid; i < nb; i += kEpiThreads) s_hist[i] = 0;
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
   constexpr int N = G * H;
   constexpr int GQ = G / EG;  // queries of a tile handled by one epilogue warpgroup
-  constexpr ScoreSmem L{N, NS, EG};
+  constexpr ScoreSmem L{N, NS, EG, EPI == kEpiScore ? G : 0};
   constexpr int ACC_COLS = N;
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32u : (2 * ACC_COLS <= 64) ? 64u
                                  : (2 * ACC_COLS <= 128) ? 128u : (2 * ACC_COLS <= 256) ? 256u : 512u;
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   float* s_w = reinterpret_cast<float*>(smem + L.off_w());
   uint64_t* s_thr = reinterpret_cast<uint64_t*>(smem + L.off_thr());
   int* s_count = reinterpret_cast<int*>(smem + L.off_count());
+  int* s_upd = reinterpret_cast<int*>(smem + L.off_upd());
   int* s_half = reinterpret_cast<int*>(smem + L.off_half());
   const uint32_t bar0 = sbase + L.off_bars();
   const uint32_t bar_q_full = bar0, bar_q_empty = bar0 + 8;
@@ -548,7 +551,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const int q_lo = e * GQ;
-    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + L.off_hist()) + e * 2048;
+    uint32_t* s_qh = reinterpret_cast<uint32_t*>(smem + L.off_hist());  // [G][kHistBins]
     int* s_misc = reinterpret_cast<int*>(smem + L.off_misc()) + e * 32;
     uint64_t* s_wred = reinterpret_cast<uint64_t*>(s_misc + 8);  // [4] lo, [4] hi per warp
     int* s_wcnt = reinterpret_cast<int*>(smem + L.off_wcnt());
@@ -558,8 +561,10 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     for (int u = u_begin; ok && u < u_end; u += u_step) {
       const Unit U = unit_geometry<G>(p, u, H);
       epi_sync(bar);
+      for (int i = etid; i < GQ * kHistBins; i += kEpiThreads) s_qh[q_lo * kHistBins + i] = 0u;
       if (etid < GQ) {
         const int qq = q_lo + etid;
+        s_upd[qq] = 0;
         s_count[qq] = 0;
         s_thr[qq] = (p.init_thr && qq < U.rows) ? p.init_thr[U.row0 + qq] : 0ull;
         s_half[qq] = 0;
@@ -654,15 +659,17 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
                             static_cast<size_t>(half[i]) * lay.half_recs() + lay.region_off(1 + quarter);
             reg[cnt[i] + __popc(bal & lt_mask)] = rec;
             const uint32_t code = static_cast<uint32_t>(rec >> 32);
+            atomicAdd(&s_qh[qq * kHistBins + (code >> kHistShift)], 1u);
             rlo[i] = min(rlo[i], code);
             rhi[i] = max(rhi[i], code);
           }
           cnt[i] += __popc(bal);
         }
-        // every 4th tile (and at the unit's end) the warpgroup publishes its
-        // append counts and compacts the buffers that could overflow within
-        // the next 4 tiles (a warp appends at most 32 records per query per tile)
-        if (((t - U.tile_lo) & 3) != 3 && t + 1 != U.tile_hi) continue;
+        // every kCheckTiles-th tile (and at the unit's end) the warpgroup
+        // publishes its append counts, raises each row's admission threshold
+        // from the row's score-code histogram, and compacts buffers that
+        // could overflow before the next check
+        if (((t - U.tile_lo) % kCheckTiles) != kCheckTiles - 1 && t + 1 != U.tile_hi) continue;
         if (lane == 0) {
 #pragma unroll
           for (int i = 0; i < GQ; ++i) s_wcnt[(q_lo + i) * 4 + quarter] = cnt[i];
@@ -671,11 +678,80 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
+          uint32_t* qh = s_qh + qq * kHistBins;
           bool full = false;
+          int total = s_count[qq];
 #pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) full = full || (s_wcnt[qq * 4 + w2] > lay.app_cap - 4 * 32);
-          if (full) {
-            // reduce the lanes' record ranges, then compact
+          for (int w2 = 0; w2 < 4; ++w2) {
+            full = full || (s_wcnt[qq * 4 + w2] > lay.app_cap - kCheckTiles * 32);
+            total += s_wcnt[qq * 4 + w2];
+          }
+          // The histogram counts exactly the buffered records.  With at least
+          // topk of them in bins >= B, a later key whose score code lies below
+          // bin B is beaten by topk records and can never be selected.
+          int kept_above = 0;
+          if (total >= p.topk && (full || total - s_upd[qq] >= 256)) {
+            epi_find_bucket(qh, kHistBins, 0, p.topk, etid, s_misc + 4, s_misc + 1, bar);
+            const uint64_t t_new = static_cast<uint64_t>(static_cast<uint32_t>(s_misc[1]) << kHistShift) << 32;
+            kept_above = s_misc[2] + s_misc[3];
+            epi_sync(bar);
+            if (etid == 0) {
+              if (t_new > s_thr[qq]) s_thr[qq] = t_new;
+              s_upd[qq] = total;
+            }
+            epi_sync(bar);
+          }
+          if (!full) continue;
+          const int half_q = s_half[qq];
+          uint64_t* qbuf = cand_unit + static_cast<size_t>(qq) * lay.query_recs();
+          const uint64_t thr_q = s_thr[qq];
+          if (kept_above <= lay.keep_cap) {
+            // one copy pass: keep the records at or above the threshold
+            const uint64_t* src = qbuf + static_cast<size_t>(half_q) * lay.half_recs();
+            uint64_t* dst = qbuf + static_cast<size_t>(half_q ^ 1) * lay.half_recs();
+            if (etid == 0) s_misc[0] = 0;
+            epi_sync(bar);
+#pragma unroll 1
+            for (int r = 0; r < 5; ++r) {
+              const uint64_t* sp = src + lay.region_off(r);
+              const int n = (r == 0) ? s_count[qq] : s_wcnt[qq * 4 + r - 1];
+              for (int base = 0; base < n; base += 8 * kEpiThreads) {
+                uint64_t v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const int idx = base + j * kEpiThreads + etid;
+                  v[j] = idx < n ? sp[idx] : 0ull;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const int idx = base + j * kEpiThreads + etid;
+                  const bool keep = (idx < n) && (v[j] >= thr_q);
+                  const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+                  if (kb) {
+                    int pos = 0;
+                    if (lane == 0) pos = atomicAdd(&s_misc[0], __popc(kb));
+                    pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+                    const int at2 = pos + __popc(kb & lt_mask);
+                    if (keep && at2 < lay.keep_cap) dst[at2] = v[j];
+                  }
+                }
+              }
+            }
+            epi_sync(bar);
+            // records below the threshold are gone: clear their bins
+            const uint32_t b_thr = static_cast<uint32_t>(thr_q >> (32 + kHistShift));
+            for (int bb = etid; bb < kHistBins; bb += kEpiThreads)
+              if (static_cast<uint32_t>(bb) < b_thr) qh[bb] = 0u;
+            if (etid == 0) {
+              s_count[qq] = min(s_misc[0], lay.keep_cap);
+#pragma unroll
+              for (int r = 0; r < 4; ++r) s_wcnt[qq * 4 + r] = 0;
+              s_half[qq] = half_q ^ 1;
+            }
+            epi_sync(bar);
+          } else {
+            // too many records share the threshold's bin: exact radix fallback
+            // (10-bit digits in the histogram array), then rebuild the histogram
             uint64_t lo = static_cast<uint64_t>(__reduce_min_sync(0xFFFFFFFFu, rlo[i])) << 32;
             uint64_t hi = (static_cast<uint64_t>(__reduce_max_sync(0xFFFFFFFFu, rhi[i])) << 32) | 0xFFFFFFFFull;
             if (lane == 0) {
@@ -688,13 +764,22 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
               lo = s_wred[w2] < lo ? s_wred[w2] : lo;
               hi = s_wred[4 + w2] > hi ? s_wred[4 + w2] : hi;
             }
-            if (thr[i] > 0ull) lo = thr[i];  // every buffered record is >= the threshold
-            epi_compact(cand_unit + static_cast<size_t>(qq) * lay.query_recs(), lay, qq, p.topk, etid,
-                        s_hist, s_thr, s_count, s_wcnt, s_half, s_misc, lo, hi, bar);
-            cnt[i] = 0;
-            rlo[i] = 0xFFFFFFFFu;
+            if (thr_q > lo) lo = thr_q;  // every buffered record is >= the threshold
+            epi_sync(bar);
+            epi_compact(qbuf, lay, qq, p.topk, etid, qh, s_thr, s_count, s_wcnt, s_half, s_misc, lo, hi, bar);
+            for (int bb = etid; bb < kHistBins; bb += kEpiThreads) qh[bb] = 0u;
+            epi_sync(bar);
+            const uint64_t* kept = qbuf + static_cast<size_t>(s_half[qq]) * lay.half_recs();
+            const int nk = s_count[qq];
+            for (int idx = etid; idx < nk; idx += kEpiThreads)
+              atomicAdd(&qh[static_cast<uint32_t>(kept[idx] >> 32) >> kHistShift], 1u);
+            epi_sync(bar);
             rhi[i] = static_cast<uint32_t>(hi >> 32);
           }
+          if (etid == 0) s_upd[qq] = s_count[qq];
+          cnt[i] = 0;
+          rlo[i] = 0xFFFFFFFFu;
+          epi_sync(bar);
         }
       }
       if (!ok) break;
@@ -724,7 +809,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 template <int H, int G, int NS, int EG, int EPI = kEpiScore>
 static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const ScoreParams& p, int grid, cudaStream_t stream) {
-  constexpr ScoreSmem L{G * H, NS, EG};
+  constexpr ScoreSmem L{G * H, NS, EG, EPI == kEpiScore ? G : 0};
   static_assert(L.request() <= 227u * 1024u, "shared memory budget");
   auto kern = score_topk_kernel<H, G, NS, EG, EPI>;
   int dev = 0;
@@ -751,7 +836,7 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_score(int H, int G, const CUtensorMap& tq, const CUtensorMap& tk,
                          const ScoreParams& p, int grid, cudaStream_t stream) {
   if (H == 64 && G == 4) return launch_score_t<64, 4, 4, 2>(tq, tk, p, grid, stream);
-  if (H == 32 && G == 8) return launch_score_t<32, 8, 4, 2>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8) return launch_score_t<32, 8, 3, 2>(tq, tk, p, grid, stream);
   if (H == 64 && G == 1) return launch_score_t<64, 1, 6, 1>(tq, tk, p, grid, stream);
   if (H == 32 && G == 1) return launch_score_t<32, 1, 6, 1>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;
