@@ -12,8 +12,11 @@ pairs per second.
     python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
 
 Under torchrun each rank runs its own replica of the workload (different
-seed) on its own GPU; there is no collective in the data path ("scaling":
-"weak"): value = all ranks' pairs / the slowest rank's time.
+seed) on its own GPU by default; there is no collective in the data path
+("scaling": "weak"): value = all ranks' pairs / the slowest rank's time.
+With --shard rows the ranks split ONE workload instead ("scaling": "strong"):
+contiguous query-row blocks balanced by visible pairs (decode: sequence
+blocks), keys replicated, still no collective in the data path.
 """
 
 from __future__ import annotations
@@ -49,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["dense", "pruned"], default="dense",
                     help="prefill path: dense fused scoring, or DoSA certified pruning")
+    ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
+                    help="N>1: independent replicas per rank (weak) or one workload split by rows (strong)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -230,6 +235,8 @@ def main():
     import torch.distributed as dist
 
     import sparse_attention_token_03_b200 as dsa
+    from sparse_attention_token_03_b200.shard import (max_over_ranks, row_shards, sequence_shards,
+                                                      shard_pairs, sum_over_ranks)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -242,7 +249,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    seed = wl.seed + 7919 * rank
+    sharded = args.shard == "rows" and world > 1
+    seed = wl.seed + (0 if sharded else 7919 * rank)
     pruned = args.path == "pruned"
     if pruned and (wl.kind != "prefill" or wl.n_seed == 0):
         raise SystemExit(f"--path pruned needs a chunked prefill workload with a seed set, not {wl.name}")
@@ -250,13 +258,31 @@ def main():
         x = make_prefill(wl, seed=seed, with_anchor=pruned)
     else:
         x = make_decode(wl, seed=seed)
+    q_off = wl.q_offset
+    if sharded:
+        # this rank's block of query rows (decode: sequences) of the one workload
+        if wl.kind == "prefill":
+            b, e = row_shards(wl.T_q, wl.q_offset, world)[rank]
+            pairs = shard_pairs(wl.T_q, wl.q_offset, (b, e))
+            q_off = wl.q_offset + b
+        else:
+            b, e = sequence_shards(x["seq_len"], world)[rank]
+            x["k"] = x["k"][b:e]
+            x["seq_len"] = x["seq_len"][b:e]
+            pairs = int(x["seq_len"].sum())
+        if e <= b:
+            raise SystemExit(f"--shard rows: rank {rank} has no rows of {wl.name}")
+        x["q"], x["w"] = x["q"][b:e], x["w"][b:e]
+    else:
+        pairs = wl.visible_pairs
+    total_pairs = sum_over_ranks(pairs, dev) if world > 1 else pairs
 
     def to_dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
     q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
     w = torch.from_numpy(x["w"]).to(dev)
-    rows = wl.T_q if wl.kind == "prefill" else wl.B
+    rows = x["q"].shape[0]
     out_idx = torch.empty((rows, wl.topk), dtype=torch.int32, device=dev)
     out_score = torch.empty((rows, wl.topk), dtype=torch.float32, device=dev)
     filter_stats = None
@@ -273,34 +299,33 @@ def main():
         rnd = random_distinct_keys(seed + 1, 0, wl.q_offset, wl.n_seed - wl.n_anchor, exclude=anchor)
         seeds = torch.from_numpy(np.concatenate([anchor, rnd]).astype(np.int32)).to(dev)
         del ka
-        ws = torch.empty(dsa.dsa_index_prefill_pruned_workspace_bytes(wl.T_q, wl.T_k, wl.H, wl.d, wl.topk,
+        ws = torch.empty(dsa.dsa_index_prefill_pruned_workspace_bytes(rows, wl.T_k, wl.H, wl.d, wl.topk,
                                                                       wl.n_seed),
                          dtype=torch.uint8, device=dev)
-        _, _, filter_stats = dsa.dsa_index_prefill_pruned(q, w, k, wl.q_offset, wl.topk, seeds,
+        _, _, filter_stats = dsa.dsa_index_prefill_pruned(q, w, k, q_off, wl.topk, seeds,
                                                           out_idx=out_idx, out_score=out_score,
                                                           workspace=ws, stats=True)
 
         def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score):
-            dsa.dsa_index_prefill_pruned(qq, ww, kk, wl.q_offset, wl.topk, seeds, out_idx=oi,
+            dsa.dsa_index_prefill_pruned(qq, ww, kk, q_off, wl.topk, seeds, out_idx=oi,
                                          out_score=osc, workspace=ws)
         n_kernels = 12
     elif wl.kind == "prefill":
-        ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(wl.T_q, wl.T_k, wl.H, wl.d, wl.topk),
+        ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(rows, wl.T_k, wl.H, wl.d, wl.topk),
                          dtype=torch.uint8, device=dev)
 
         def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score):
-            dsa.dsa_index_prefill(qq, ww, kk, wl.q_offset, wl.topk, out_idx=oi, out_score=osc,
+            dsa.dsa_index_prefill(qq, ww, kk, q_off, wl.topk, out_idx=oi, out_score=osc,
                                   workspace=ws)
         n_kernels = 2
     else:
         seq_len = torch.from_numpy(x["seq_len"]).to(dev)
-        ws = torch.empty(dsa.dsa_index_decode_workspace_bytes(wl.B, wl.t_cap, wl.H, wl.d, wl.topk),
+        ws = torch.empty(dsa.dsa_index_decode_workspace_bytes(rows, wl.t_cap, wl.H, wl.d, wl.topk),
                          dtype=torch.uint8, device=dev)
 
         def step(qq=q, ww=w, kk=k, oi=out_idx, osc=out_score, sl=seq_len):
             dsa.dsa_index_decode(qq, ww, kk, sl, wl.topk, out_idx=oi, out_score=osc, workspace=ws)
         n_kernels = 3
-    pairs = wl.visible_pairs
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -338,12 +363,8 @@ def main():
     dsa.dsa_profile_enable(False)
     status = dsa.dsa_index_device_status(ws)
 
-    ms_step = float(np.mean(step_ms))
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * pairs / (ms_step * 1e-3)
+    ms_step = max_over_ranks(float(np.mean(step_ms)), dev)
+    value = total_pairs / (ms_step * 1e-3)
 
     # ---- roofline of the dominant kernel (the fused score + Top-k kernel)
     pk, pk_src = peaks()
@@ -389,7 +410,7 @@ def main():
             extra["sl"] = torch.from_numpy(x["seq_len"]).pin_memory()
             dsl = torch.empty_like(seq_len)
         dq, dk, dw = torch.empty_like(q), torch.empty_like(k), torch.empty_like(w)
-        h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + (wl.B * 4 if wl.kind == "decode" else 0)
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + (rows * 4 if wl.kind == "decode" else 0)
         d2h = hoi.numel() * 4 + hos.numel() * 4
         n_e2e = max(3, min(args.steps, 20))
         e_ms = []
@@ -412,12 +433,8 @@ def main():
             ev1.synchronize()
             if i >= 2:
                 e_ms.append(ev0.elapsed_time(ev1))
-        em = float(np.mean(e_ms))
-        if world > 1:
-            t = torch.tensor([em], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            em = float(t.item())
-        e2e = {"value": world * pairs / (em * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
+        em = max_over_ranks(float(np.mean(e_ms)), dev)
+        e2e = {"value": total_pairs / (em * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": em}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
@@ -433,9 +450,11 @@ def main():
             "metric": "indexer causal q.k pairs/s" + (" (effective, DoSA)" if pruned else ""),
             "value": value, "unit": "pairs/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
-                                                 parallelism=f"replicas x{world}", path=args.path),
+            "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
+                           parallelism=(f"row blocks x{world}" if sharded else f"replicas x{world}"),
+                           path=args.path),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": n_kernels * args.steps, "clocks": clocks, "device_status": status,
             "kernel_ms": {n: float(np.mean(v)) for n, v in kern_ms.items()},
