@@ -22,6 +22,8 @@ namespace dsa {
 namespace {
 
 constexpr int kStageRecs = 7680;  // candidates of a row staged in shared memory (60 KB)
+constexpr int kWinCap = 4096;     // records in the boundary bucket and above it (32 KB)
+constexpr int kRankMax = 256;     // largest bucket ranked by counting
 
 __device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_t digit) {
   if (valid) atomicAdd(&hist[digit], 1u);
@@ -140,21 +142,32 @@ __device__ __forceinline__ void sort2048_desc(uint64_t (&v)[8], uint64_t* s_x) {
 }  // namespace
 
 // One CTA of 256 threads per output row.
+//
+// Staged rows (the usual case) take one counting pass: digit(r) =
+// (r - lo) >> shift over the row's record range [lo, hi] (2048 buckets,
+// ascending in the record order), a descending prefix scan of the bucket
+// counts, which also finds the bucket holding the m-th record, a scatter of
+// every record in that bucket or above it into bucket order, and a rank
+// count inside each bucket that puts each winner straight at its final
+// position.  Rows whose candidates do not fit the staging buffer, or whose
+// records crowd more than kRankMax into one bucket, take the radix-select +
+// bitonic-sort path instead.
 template <int NT>
 __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   static_assert(NT == 256, "the sort layout assumes 256 threads x 8 records");
   extern __shared__ __align__(16) uint64_t s_dyn[];
   uint64_t* s_rec = s_dyn;               // [kStageRecs] staged candidates (0 = empty slot)
-  uint64_t* s_win = s_dyn + kStageRecs;  // [2048] winners / sort exchange
-  __shared__ uint32_t s_hist[2048];
+  uint64_t* s_win = s_dyn + kStageRecs;  // [kWinCap] winners in bucket order / sort exchange
+  __shared__ __align__(16) uint32_t s_hist[2048];
+  __shared__ __align__(16) uint32_t s_cur[2048];
   __shared__ int s_scratch[NT / 32];
   __shared__ int s_res[4];
-  __shared__ int s_n, s_staged, s_pos;
+  __shared__ int s_n, s_staged, s_pos, s_maxc;
   __shared__ unsigned long long s_lo, s_hi;
   __shared__ __align__(8) uint64_t s_bar;
 
   const int64_t row = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   if (p.row_flags && p.row_flags[row] == 0) return;  // row already exact
   const RowUnits R = row_units(p, row);
   const int G = (p.mode == kModeDecode) ? 1 : p.G;
@@ -177,19 +190,55 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   };
   const int n_seg = 5 * R.n_u + (p.extra_rec ? 1 : 0);
 
-  if (tid == 0) {
+  // warp 0 sizes the segments (one lane per segment, a warp scan for the
+  // staging offsets) and, when they fit, issues one bulk copy per segment
+  // into consecutive 16-byte aligned slots
+  if (wid == 0) {
     int n = 0, staged = 0;
-    for (int sg = 0; sg < n_seg; ++sg) {
-      int c;
-      segment(sg, c);
+    for (int base = 0; base < n_seg; base += 32) {
+      int c = 0;
+      if (base + lane < n_seg) segment(base + lane, c);
+      int c2 = (c + 1) & ~1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+        c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
+      }
       n += c;
-      staged += (c + 1) & ~1;
+      staged += c2;
     }
-    s_n = n;
-    s_staged = staged;
-    s_pos = 0;
-    s_lo = ~0ull;
-    s_hi = 0ull;
+    if (lane == 0) {
+      s_n = n;
+      s_staged = staged;
+      s_pos = 0;
+      s_maxc = 0;
+      s_lo = ~0ull;
+      s_hi = 0ull;
+    }
+    if (staged <= kStageRecs && n > 0) {
+      const uint32_t bar = smem_u32(&s_bar);
+      if (lane == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(staged) * 8u);
+      }
+      __syncwarp();
+      int off = 0;
+      for (int base = 0; base < n_seg; base += 32) {
+        int c = 0;
+        const uint64_t* src = nullptr;
+        if (base + lane < n_seg) src = segment(base + lane, c);
+        const int c2 = (c + 1) & ~1;
+        int incl = c2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (c2 > 0) bulk_load(smem_u32(s_rec + off + incl - c2), src, static_cast<uint32_t>(c2) * 8u, bar);
+        off += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+    }
   }
   __syncthreads();
   const int n = s_n;
@@ -198,62 +247,148 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   const int n_st = staged ? s_staged : 0;
 
   if (staged && n > 0) {
-    // one bulk copy per segment into consecutive 16-byte aligned slots
-    const uint32_t bar = smem_u32(&s_bar);
-    if (tid == 0) {
-      mbar_init(bar, 1);
-      fence_mbar_init();
-      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(n_st) * 8u);
-      int off = 0;
-      for (int sg = 0; sg < n_seg; ++sg) {
-        int c;
-        const uint64_t* src = segment(sg, c);
-        const int c2 = (c + 1) & ~1;
-        if (c2 > 0) bulk_load(smem_u32(s_rec + off), src, static_cast<uint32_t>(c2) * 8u, bar);
-        off += c2;
-      }
-    }
-    __syncthreads();
     volatile int never = 0;
-    mbar_wait(bar, 0, &never, p.err);
-    __syncthreads();
-    if (tid == 0) {  // blank the padding slot after each odd-sized segment
+    mbar_wait(smem_u32(&s_bar), 0, &never, p.err);
+    __syncwarp();
+    if (wid == 0) {  // blank the padding slot after each odd-sized segment
       int off = 0;
-      for (int sg = 0; sg < n_seg; ++sg) {
-        int c;
-        segment(sg, c);
-        if (c & 1) s_rec[off + c] = 0ull;
-        off += (c + 1) & ~1;
+      for (int base = 0; base < n_seg; base += 32) {
+        int c = 0;
+        if (base + lane < n_seg) segment(base + lane, c);
+        const int c2 = (c + 1) & ~1;
+        int incl = c2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (c & 1) s_rec[off + incl - 1] = 0ull;
+        off += __shfl_sync(0xFFFFFFFFu, incl, 31);
       }
     }
     __syncthreads();
   }
 
+  const size_t o = static_cast<size_t>(row) * p.topk;
+  const size_t orec = static_cast<size_t>(row) * p.rec_stride;
+  auto put = [&](int i, uint64_t r) {  // position i of the row's output; r = 0 pads
+    const bool ok = r != 0ull;
+    if (p.out_idx) p.out_idx[o + i] = ok ? static_cast<int32_t>(record_key(r)) : -1;
+    if (p.out_score) p.out_score[o + i] = ok ? record_score(r) : -INFINITY;
+    if (p.out_rec) p.out_rec[orec + i] = r;
+    if (p.out_kth && i == m - 1) p.out_kth[row] = record_score(r);
+  };
+  if (p.out_kth && m == 0 && tid == 0) p.out_kth[row] = -INFINITY;
+
+  // ---- counting path
+  bool done = false;
+  if (staged && m > 0) {
+    uint64_t lo = ~0ull, hi = 0ull;
+    for (int i = tid; i < n_st; i += NT) {
+      const uint64_t r = s_rec[i];
+      if (r != 0ull) {
+        lo = r < lo ? r : lo;
+        hi = r > hi ? r : hi;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+      lo = l2 < lo ? l2 : lo;
+      hi = h2 > hi ? h2 : hi;
+    }
+    for (int i = tid; i < 2048; i += NT) s_hist[i] = 0u;
+    if (lane == 0) {
+      atomicMin(&s_lo, static_cast<unsigned long long>(lo));
+      atomicMax(&s_hi, static_cast<unsigned long long>(hi));
+    }
+    __syncthreads();
+    const uint64_t rlo = s_lo;
+    const uint64_t span = s_hi - rlo;
+    const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 11);  // span >> shift < 2048
+    auto digit = [&](uint64_t r) { return static_cast<uint32_t>((r - rlo) >> shift); };
+    for (int i = tid; i < n_st; i += NT) {
+      const uint64_t r = s_rec[i];
+      if (r != 0ull) atomicAdd(&s_hist[digit(r)], 1u);
+    }
+    __syncthreads();
+    // descending exclusive scan: thread t owns buckets 2047-8t down to 2040-8t
+    const uint4 ha = reinterpret_cast<const uint4*>(s_hist)[(2040 - 8 * tid) >> 2];
+    const uint4 hb = reinterpret_cast<const uint4*>(s_hist)[(2044 - 8 * tid) >> 2];
+    const uint32_t c[8] = {hb.w, hb.z, hb.y, hb.x, ha.w, ha.z, ha.y, ha.x};
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sum += c[j];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) s_scratch[wid] = static_cast<int>(incl);
+    __syncthreads();
+    uint32_t run = incl - sum;
+    for (int w2 = 0; w2 < wid; ++w2) run += static_cast<uint32_t>(s_scratch[w2]);
+    uint32_t ex[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ex[j] = run;
+      const int d = 2047 - 8 * tid - j;
+      if (c[j] > 0u && run <= static_cast<uint32_t>(m - 1) && static_cast<uint32_t>(m - 1) < run + c[j]) {
+        s_res[0] = d;
+        s_res[1] = static_cast<int>(run);
+        s_res[2] = static_cast<int>(c[j]);
+      }
+      run += c[j];
+    }
+    reinterpret_cast<uint4*>(s_cur)[(2040 - 8 * tid) >> 2] = make_uint4(ex[7], ex[6], ex[5], ex[4]);
+    reinterpret_cast<uint4*>(s_cur)[(2044 - 8 * tid) >> 2] = make_uint4(ex[3], ex[2], ex[1], ex[0]);
+    __syncthreads();
+    const int B = s_res[0], above = s_res[1], cntB = s_res[2];
+    uint32_t mc = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (2047 - 8 * tid - j >= B) mc = c[j] > mc ? c[j] : mc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint32_t v = __shfl_xor_sync(0xFFFFFFFFu, mc, off);
+      mc = v > mc ? v : mc;
+    }
+    if (lane == 0) atomicMax(&s_maxc, static_cast<int>(mc));
+    __syncthreads();
+    const int nw = above + cntB;  // records in bucket B and above
+    if (nw <= kWinCap && s_maxc <= kRankMax) {
+      for (int i = tid; i < n_st; i += NT) {
+        const uint64_t r = s_rec[i];
+        if (r == 0ull) continue;
+        const uint32_t d = digit(r);
+        if (static_cast<int>(d) >= B) s_win[atomicAdd(&s_cur[d], 1u)] = r;
+      }
+      __syncthreads();
+      // s_cur[d] is now the end of bucket d; rank each record inside its bucket
+      for (int i = tid; i < nw; i += NT) {
+        const uint64_t r = s_win[i];
+        const uint32_t d = digit(r);
+        const int end = static_cast<int>(s_cur[d]), beg = end - static_cast<int>(s_hist[d]);
+        int rank = 0;
+        for (int j = beg; j < end; ++j) rank += (s_win[j] > r) ? 1 : 0;
+        if (beg + rank < m) put(beg + rank, r);
+      }
+      for (int i = m + tid; i < p.topk; i += NT) put(i, 0ull);
+      done = true;
+    }
+    __syncthreads();
+  }
+  if (done) return;
+
+  // ---- radix-select + bitonic-sort path
   uint64_t thr = 1;  // records are >= 1: keeps all
   if (m > 0 && m < n) {
     uint64_t prefix = 0;
     int pbits = 0, above = 0;
     if (staged) {
       // start the digits at the highest bit in which the records differ
-      uint64_t lo = ~0ull, hi = 0ull;
-      for (int i = tid; i < n_st; i += NT) {
-        const uint64_t r = s_rec[i];
-        if (r != 0ull) {
-          lo = r < lo ? r : lo;
-          hi = r > hi ? r : hi;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, o), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
-        lo = l2 < lo ? l2 : lo;
-        hi = h2 > hi ? h2 : hi;
-      }
-      if ((tid & 31) == 0) {
-        atomicMin(&s_lo, static_cast<unsigned long long>(lo));
-        atomicMax(&s_hi, static_cast<unsigned long long>(hi));
-      }
-      __syncthreads();
+      // (s_lo / s_hi were reduced by the counting path)
       const uint64_t diff = s_lo ^ s_hi;  // non-zero: records are distinct
       pbits = __clzll(static_cast<long long>(diff));
       prefix = pbits > 0 ? (s_hi >> (64 - pbits)) : 0ull;
@@ -312,7 +447,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
       if (bal) {
         int pos = 0;
-        if ((tid & 31) == 0) pos = atomicAdd(&s_pos, __popc(bal));
+        if (lane == 0) pos = atomicAdd(&s_pos, __popc(bal));
         pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
         const int at = pos + __popc(bal & lanemask_lt());
         if (keep && at < kMaxTopk) s_win[at] = r;
@@ -338,30 +473,17 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   }
   __syncthreads();
   sort2048_desc(v, s_win);
-  const size_t o = static_cast<size_t>(row) * p.topk;
-  const size_t orec = static_cast<size_t>(row) * p.rec_stride;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int i = 8 * tid + s;
-    if (i < p.topk) {
-      const bool ok = i < m;
-      if (p.out_idx) p.out_idx[o + i] = ok ? static_cast<int32_t>(record_key(v[s])) : -1;
-      if (p.out_score) p.out_score[o + i] = ok ? record_score(v[s]) : -INFINITY;
-      if (p.out_rec) p.out_rec[orec + i] = ok ? v[s] : 0ull;
-    }
-  }
-  if (p.out_kth) {
-    if (m == 0 && tid == 0) p.out_kth[row] = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < 8; ++s)
-      if (8 * tid + s == m - 1) p.out_kth[row] = record_score(v[s]);
+    if (i < p.topk) put(i, i < m ? v[s] : 0ull);
   }
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   if (p.n_rows <= 0) return cudaSuccess;
   constexpr int NT = kSelectThreads;
-  const size_t smem = (kStageRecs + kMaxTopk) * sizeof(uint64_t);
+  const size_t smem = (kStageRecs + kWinCap) * sizeof(uint64_t);
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
