@@ -143,13 +143,13 @@ __device__ __forceinline__ void sort2048_desc(uint64_t (&v)[8], uint64_t* s_x) {
 
 // One CTA of 256 threads per output row.
 //
-// Staged rows (the usual case) take one counting pass: digit(r) =
-// (r - lo) >> shift over the row's record range [lo, hi] (2048 buckets,
-// ascending in the record order), a descending prefix scan of the bucket
+// Staged rows (the usual case) take one counting pass: a 2048-bucket digit
+// of each record that never decreases along the record order (linear in the
+// score over the row's score range), a descending prefix scan of the bucket
 // counts, which also finds the bucket holding the m-th record, a scatter of
 // every record in that bucket or above it into bucket order, and a rank
-// count inside each bucket that puts each winner straight at its final
-// position.  Rows whose candidates do not fit the staging buffer, or whose
+// count inside each bucket that gives each winner its final position (the
+// row's output is then written in order).  Rows whose candidates do not fit the staging buffer, or whose
 // records crowd more than kRankMax into one bucket, take the radix-select +
 // bitonic-sort path instead.
 template <int NT>
@@ -303,10 +303,20 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       atomicMax(&s_hi, static_cast<unsigned long long>(hi));
     }
     __syncthreads();
+    // bucket of a record: linear in its score between the row's smallest and
+    // largest score (any digit that never decreases along the record order
+    // works; a linear one spreads the winners evenly), or, when that range is
+    // zero or not finite, the top 11 bits of (record - smallest record)
     const uint64_t rlo = s_lo;
     const uint64_t span = s_hi - rlo;
     const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 11);  // span >> shift < 2048
-    auto digit = [&](uint64_t r) { return static_cast<uint32_t>((r - rlo) >> shift); };
+    const float smin = record_score(rlo), srange = record_score(s_hi) - smin;
+    const float scale = 2047.0f / srange;
+    const bool lin = srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f;
+    auto digit = [&](uint64_t r) {
+      if (lin) return min(2047u, static_cast<uint32_t>((record_score(r) - smin) * scale));
+      return static_cast<uint32_t>((r - rlo) >> shift);
+    };
     for (int i = tid; i < n_st; i += NT) {
       const uint64_t r = s_rec[i];
       if (r != 0ull) atomicAdd(&s_hist[digit(r)], 1u);
@@ -365,16 +375,18 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
         if (static_cast<int>(d) >= B) s_win[atomicAdd(&s_cur[d], 1u)] = r;
       }
       __syncthreads();
-      // s_cur[d] is now the end of bucket d; rank each record inside its bucket
+      // s_cur[d] is now the end of bucket d; rank each record inside its
+      // bucket and place the winners in order in the (now free) staging buffer
       for (int i = tid; i < nw; i += NT) {
         const uint64_t r = s_win[i];
         const uint32_t d = digit(r);
         const int end = static_cast<int>(s_cur[d]), beg = end - static_cast<int>(s_hist[d]);
         int rank = 0;
         for (int j = beg; j < end; ++j) rank += (s_win[j] > r) ? 1 : 0;
-        if (beg + rank < m) put(beg + rank, r);
+        if (beg + rank < m) s_rec[beg + rank] = r;
       }
-      for (int i = m + tid; i < p.topk; i += NT) put(i, 0ull);
+      __syncthreads();
+      for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_rec[i] : 0ull);
       done = true;
     }
     __syncthreads();
