@@ -118,6 +118,7 @@ int check_shape(int H, int d, int topk) {
 // ----------------------------------------------------------------- prefill
 struct PrefillPlan {
   int G, n_groups, S, n_units, grid;
+  int eg;  // epilogue warpgroups of the fused kernel (2 or 4)
   CandLayout lay;
   size_t off_meta, off_cand, bytes;
 };
@@ -137,6 +138,13 @@ PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H,
     P.S = std::min(P.S, 64);
   }
   P.n_units = P.n_groups * P.S;
+  // Epilogue width: four warpgroups (one query each at H = 64) hide the
+  // admission work of units whose keys are few per selected record; with
+  // many keys per record admissions are rare, the head sums dominate and two
+  // warpgroups with the head weights in registers issue fewer instructions.
+  const double unit_keys = (static_cast<double>(std::max<int64_t>(q_offset_hint, 0)) +
+                            0.5 * static_cast<double>(T_q + 1)) / P.S;
+  P.eg = unit_keys >= static_cast<double>(kWideKeysPerRecord) * topk ? 2 : 4;
   P.lay = cand_layout(topk);
   P.grid = std::max(1, std::min(sms, P.n_units));
   size_t off = 256;  // device status word
@@ -243,7 +251,7 @@ int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const
   sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = dp.err;
-  if ((e = launch_score(H, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  if ((e = launch_score(H, 1, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
   if (profile) prof_mark(st, "score_topk");
 
   SelectParams se{};
@@ -413,7 +421,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = reinterpret_cast<uint32_t*>(ws);
-  if ((e = launch_score(H, P.G, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  if ((e = launch_score(H, P.G, P.eg, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
   prof_mark(st, "score_topk");
 
   SelectParams se{};
@@ -518,7 +526,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     s1.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + P.seed.off_cand));
     s1.meta = reinterpret_cast<int32_t*>(at(P.off_cand + P.seed.off_meta));
     s1.err = err;
-    if ((e = launch_score(H, P.seed.G, tq, tks, s1, P.seed.grid, st)) != cudaSuccess)
+    if ((e = launch_score(H, P.seed.G, P.seed.eg, tq, tks, s1, P.seed.grid, st)) != cudaSuccess)
       return cuda_fail(e, "seed score launch");
     prof_mark(st, "seed_score");
     SelectParams s2{};
@@ -613,7 +621,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     s4.surv_stride = P.cap_row;
     s4.k_gather = k;
     s4.init_thr = reinterpret_cast<const uint64_t*>(at(P.off_init_thr));
-    if ((e = launch_score(H, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
+    if ((e = launch_score(H, 1, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
     prof_mark(st, "refine");
     SelectParams s5{};
     s5.mode = kModeDecode;
@@ -653,7 +661,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     s6.row_flags = reinterpret_cast<const int32_t*>(at(P.off_row_flags));
     CUtensorMap tqd;
     if ((rc = make_tmap(&tqd, q, T_q * H, P.dense.G * H)) != DSA_OK) return rc;
-    if ((e = launch_score(H, P.dense.G, tqd, tk, s6, P.dense.grid, st)) != cudaSuccess)
+    if ((e = launch_score(H, P.dense.G, P.dense.eg, tqd, tk, s6, P.dense.grid, st)) != cudaSuccess)
       return cuda_fail(e, "recovery launch");
     SelectParams s7{};
     s7.mode = kModePrefill;

@@ -21,16 +21,26 @@ constexpr int kTileKeys = 128;   // keys per MMA tile (M)
 constexpr int kMaxTopk = 2048;   // largest supported k
 constexpr int kEpiThreads = 128; // threads of one epilogue warpgroup
 // Score kernel block: one epilogue warpgroup runs after a producer warp and an
-// MMA warp (6 warps); two epilogue warpgroups run after a whole control
-// warpgroup (producer, MMA, two idle warps) so that registers can be moved
-// between warpgroups with setmaxnreg (12 warps).
+// MMA warp (6 warps); two or four epilogue warpgroups run after a whole
+// control warpgroup (producer, MMA, two idle warps) so that registers can be
+// moved between warpgroups with setmaxnreg (12 or 20 warps).
 __host__ __device__ constexpr int score_epi_warp0(int eg) { return eg == 1 ? 2 : 4; }
 __host__ __device__ constexpr int score_threads(int eg) { return 32 * score_epi_warp0(eg) + kEpiThreads * eg; }
-// Register split of the 12-warp block: 168 at launch (65536 / 384 rounded to
-// 8), then 128 x 56 (control) + 256 x 224 (epilogue) = 384 x 168.
-constexpr uint32_t kRegsLaunch12 = 168, kRegsCtl12 = 56, kRegsEpi12 = 224;
-static_assert(128 * kRegsCtl12 + 256 * kRegsEpi12 == 384 * kRegsLaunch12, "register split must balance");
+// Register split with eg = 2 or 4 epilogue warpgroups: registers per thread
+// at launch (65536 / threads, rounded down to 8), then the control
+// warpgroup's and each epilogue thread's after setmaxnreg.  The split may
+// not ask for more than the block launched with: 128 x 56 + 256 x 224 =
+// 384 x 168 and 128 x 56 + 512 x 104 <= 640 x 96.
+__host__ __device__ constexpr uint32_t regs_launch(int eg) { return eg == 2 ? 168u : 96u; }
+__host__ __device__ constexpr uint32_t regs_ctl(int) { return 56u; }
+__host__ __device__ constexpr uint32_t regs_epi(int eg) { return eg == 2 ? 224u : 104u; }
+static_assert(128 * regs_ctl(2) + 256 * regs_epi(2) <= 384 * regs_launch(2), "register split (12 warps)");
+static_assert(128 * regs_ctl(4) + 512 * regs_epi(4) <= 640 * regs_launch(4), "register split (20 warps)");
+static_assert(regs_launch(2) * 384 <= 65536 && regs_launch(4) * 640 <= 65536, "launch registers");
 constexpr int kSelectThreads = 256;
+// A grouped prefill unit whose keys number at least this many times topk
+// runs the two-warpgroup epilogue, shorter ones the four-warpgroup one.
+constexpr int kWideKeysPerRecord = 256;
 
 constexpr int kMetaInts = 8;
 // Score-code histogram of a query's buffered records: bin = code >> 22
@@ -162,7 +172,8 @@ struct ScoreSmem {
   __host__ __device__ constexpr uint32_t k_stage() const { return 2u * k_sub(); }
   __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
-  // screening-plan scalars (screen): 2 KB
+  // screening-plan scalars (screen) or the head weights of the tile's queries
+  // (score epilogue with four warpgroups): 2 KB
   __host__ __device__ constexpr uint32_t off_hist() const { return off_w() + 512u * 4u; }
   __host__ __device__ constexpr uint32_t off_thr() const { return off_hist() + nqh * kHistBins * 4u; }
   // per query: base count, count at the last threshold update; per (query,
@@ -182,7 +193,7 @@ struct ScoreSmem {
 };
 
 // Launchers (defined in the .cu files).
-cudaError_t launch_score(int H, int G, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                          const ScoreParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_screen(const CUtensorMap& tmap_plan, const CUtensorMap& tmap_k, const ScoreParams& p,
                           int grid, cudaStream_t stream);

@@ -253,15 +253,44 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 // in ascending j starting from +0, combined as
 // ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)).
 // The eight chains give the epilogue enough independent work to issue every
-// cycle (one chain of H FMAs would stall on FMA latency).  head_acc16 adds
-// 16 consecutive heads (j0 .. j0+15, j0 a multiple of 16) to the chains.
-__device__ __forceinline__ void head_acc16(float (&a)[8], const uint32_t (&x)[16], const float* w) {
+// cycle (one chain of H FMAs would stall on FMA latency).
+//
+// Each step is computed as fma(w_j / 2, dot_j + |dot_j|, a_c), which equals
+// fma(w_j, max(dot_j, 0), a_c) bit for bit: dot + |dot| is exactly 2 dot or
+// +0, and w / 2 is exact for normal weights, so the product is the same real
+// number and the FMA rounds once either way.  The add (with an absolute-value
+// operand) and the FMA run on the FMA pipe, where a max would take the ALU,
+// and chains c and c+1 advance together in one paired FMA (__ffma2_rn, per
+// component the same operation as fmaf).  head_acc16 adds 16 consecutive
+// heads (j0 .. j0+15, j0 a multiple of 16) to the chains, held as pairs
+// a[c/2] = (a_c, a_c+1); wh holds the HALVED weights of those heads.
+__device__ __forceinline__ void head_acc16(float2 (&a)[4], const uint32_t (&x)[16], const float* wh) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j) a[j & 7] = fmaf(w[j], fmaxf(__uint_as_float(x[j]), 0.0f), a[j & 7]);
+  for (int j = 0; j < 16; j += 2) {
+    const float x0 = __uint_as_float(x[j]), x1 = __uint_as_float(x[j + 1]);
+    a[(j & 7) >> 1] = __ffma2_rn(make_float2(wh[j], wh[j + 1]), make_float2(x0 + fabsf(x0), x1 + fabsf(x1)),
+                                 a[(j & 7) >> 1]);
+  }
 }
-__device__ __forceinline__ float head_finish(const float (&a)[8]) {
-  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+// The same 16 heads with the halved weights read from shared memory (16-byte
+// broadcast loads; identical arithmetic).
+__device__ __forceinline__ void head_acc16_smem(float2 (&a)[4], const uint32_t (&x)[16], const float* wh) {
+  float wv[16];
+#pragma unroll
+  for (int j4 = 0; j4 < 4; ++j4) {
+    const float4 v = reinterpret_cast<const float4*>(wh)[j4];
+    wv[4 * j4 + 0] = v.x;
+    wv[4 * j4 + 1] = v.y;
+    wv[4 * j4 + 2] = v.z;
+    wv[4 * j4 + 3] = v.w;
+  }
+  head_acc16(a, x, wv);
 }
+__device__ __forceinline__ float head_finish(const float2 (&a)[4]) {
+  return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+}
+// Halved head weight as head_acc16 takes it (exact for normal weights).
+__device__ __forceinline__ float half_weight(float w) { return 0.5f * w; }
 
 // Monotone 32-bit code of an fp32 score: larger score <=> larger code.
 // -0 is folded onto +0 first.

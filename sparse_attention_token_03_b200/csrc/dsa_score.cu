@@ -259,6 +259,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
   constexpr int N = G * H;
   constexpr int GQ = G / EG;  // queries of a tile handled by one epilogue warpgroup
+  constexpr bool kWSmem = EG >= 4;  // head weights read from shared memory (register budget)
   constexpr ScoreSmem L{N, NS, EG, EPI == kEpiScore ? G : 0};
   constexpr int ACC_COLS = N;
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32u : (2 * ACC_COLS <= 64) ? 64u
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 
   if (warp < score_epi_warp0(EG)) {
    // one setmaxnreg for the whole control warpgroup
-   if constexpr (EG == 2) regs_dec<kRegsCtl12>();
+   if constexpr (EG >= 2) regs_dec<regs_ctl(EG)>();
    if (warp == 0 && p.mode == kModeRefine) {
     // ------------------------------------------------ producer (gathered keys)
     // Survivor keys are gathered row by row with 16-byte cp.async into the
@@ -468,7 +469,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     // d_neg; C carries the residual, bf16-rounding and fp32 slack terms).  A
     // visible non-seed key survives unless U < tau ("DoSA", step 2: prune only
     // when the bound is strictly below the threshold, keep when unsure).
-    if constexpr (EG == 2) regs_inc<kRegsEpi12>();
+    if constexpr (EG >= 2) regs_inc<regs_epi(EG)>();
     const int e = (warp - score_epi_warp0(EG)) >> 2;
     const int bar = 1 + e;
     const int etid = (threadIdx.x - 32 * score_epi_warp0(EG)) & (kEpiThreads - 1);
@@ -543,7 +544,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    if constexpr (EG == 2) regs_inc<kRegsEpi12>();
+    if constexpr (EG >= 2) regs_inc<regs_epi(EG)>();
     const int e = (warp - score_epi_warp0(EG)) >> 2;  // epilogue warpgroup
     const int bar = 1 + e;
     const int etid = (threadIdx.x - 32 * score_epi_warp0(EG)) & (kEpiThreads - 1);
@@ -571,21 +572,31 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int r = 0; r < 4; ++r) s_wcnt[qq * 4 + r] = 0;
       }
+      if constexpr (kWSmem) {
+        // this warpgroup's halved head weights, in shared memory for the whole unit
+        for (int i = etid; i < GQ * H; i += kEpiThreads) {
+          const int qq = q_lo + i / H;
+          s_w[q_lo * H + i] = qq < U.rows ? half_weight(__ldg(p.w + (U.row0 + qq) * H + i % H)) : 0.0f;
+        }
+      }
       epi_sync(bar);
-      // this warpgroup's head weights stay in registers for the whole unit
-      float wr[GQ][H];
+      // with one or two warpgroups, the halved head weights stay in registers
+      // for the whole unit
+      float wr[kWSmem ? 1 : GQ][kWSmem ? 1 : H];
+      if constexpr (!kWSmem) {
 #pragma unroll
-      for (int i = 0; i < GQ; ++i) {
-        const int qq = q_lo + i;
-        const float4* src = reinterpret_cast<const float4*>(p.w + (U.row0 + (qq < U.rows ? qq : 0)) * H);
+        for (int i = 0; i < GQ; ++i) {
+          const int qq = q_lo + i;
+          const float4* src = reinterpret_cast<const float4*>(p.w + (U.row0 + (qq < U.rows ? qq : 0)) * H);
 #pragma unroll
-        for (int j4 = 0; j4 < H / 4; ++j4) {
-          const float4 v = __ldg(src + j4);
-          const bool on = qq < U.rows;
-          wr[i][4 * j4 + 0] = on ? v.x : 0.0f;
-          wr[i][4 * j4 + 1] = on ? v.y : 0.0f;
-          wr[i][4 * j4 + 2] = on ? v.z : 0.0f;
-          wr[i][4 * j4 + 3] = on ? v.w : 0.0f;
+          for (int j4 = 0; j4 < H / 4; ++j4) {
+            const float4 v = __ldg(src + j4);
+            const bool on = qq < U.rows;
+            wr[i][4 * j4 + 0] = on ? half_weight(v.x) : 0.0f;
+            wr[i][4 * j4 + 1] = on ? half_weight(v.y) : 0.0f;
+            wr[i][4 * j4 + 2] = on ? half_weight(v.z) : 0.0f;
+            wr[i][4 * j4 + 3] = on ? half_weight(v.w) : 0.0f;
+          }
         }
       }
       uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * lay.query_recs();
@@ -622,7 +633,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
                               static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
         uint32_t xb[3][16];
         float score[GQ];
-        float acc[8];
+        float2 acc[4];
         tmem_ld16(trow, xb[0]);
         if (NC > 1) tmem_ld16(trow + 16, xb[1]);
         tmem_wait_ld();
@@ -632,9 +643,13 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           if (c + 2 < NC) tmem_ld16(trow + (c + 2) * 16, xb[(c + 2) % 3]);
           if (c % CPQ == 0) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.0f, 0.0f);
           }
-          head_acc16(acc, xb[c % 3], &wr[c / CPQ][(c % CPQ) * 16]);
+          if constexpr (kWSmem) {
+            head_acc16_smem(acc, xb[c % 3], s_w + (q_lo + c / CPQ) * H + (c % CPQ) * 16);
+          } else {
+            head_acc16(acc, xb[c % 3], &wr[c / CPQ][(c % CPQ) * 16]);
+          }
           if (c % CPQ == CPQ - 1) score[c / CPQ] = head_finish(acc);
           if (c + 2 < NC) tmem_wait_ld();
           // after the last load has landed, release the accumulator
@@ -819,13 +834,13 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L.request()));
     if (e != cudaSuccess) return e;
-    if constexpr (EG == 2) {
+    if constexpr (EG >= 2) {
       // the setmaxnreg split only balances if every thread launches with exactly
-      // kRegsLaunch12 registers; refuse to launch otherwise (it would never finish)
+      // regs_launch(EG) registers; refuse to launch otherwise (it would never finish)
       cudaFuncAttributes fa{};
       e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return e;
-      if (fa.numRegs != static_cast<int>(kRegsLaunch12)) return cudaErrorInvalidConfiguration;
+      if (fa.numRegs != static_cast<int>(regs_launch(EG))) return cudaErrorInvalidConfiguration;
     }
     configured[dev] = true;
   }
@@ -833,10 +848,12 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
   return cudaGetLastError();
 }
 
-cudaError_t launch_score(int H, int G, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tq, const CUtensorMap& tk,
                          const ScoreParams& p, int grid, cudaStream_t stream) {
-  if (H == 64 && G == 4) return launch_score_t<64, 4, 4, 2>(tq, tk, p, grid, stream);
-  if (H == 32 && G == 8) return launch_score_t<32, 8, 3, 2>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 4 && eg == 4) return launch_score_t<64, 4, 4, 4>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 4 && eg == 2) return launch_score_t<64, 4, 4, 2>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8 && eg == 4) return launch_score_t<32, 8, 3, 4>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8 && eg == 2) return launch_score_t<32, 8, 3, 2>(tq, tk, p, grid, stream);
   if (H == 64 && G == 1) return launch_score_t<64, 1, 6, 1>(tq, tk, p, grid, stream);
   if (H == 32 && G == 1) return launch_score_t<32, 1, 6, 1>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;

@@ -24,6 +24,7 @@ namespace {
 constexpr int kStageRecs = 7680;  // candidates of a row staged in shared memory (60 KB)
 constexpr int kWinCap = 4096;     // records in the boundary bucket and above it (32 KB)
 constexpr int kRankMax = 256;     // largest bucket ranked by counting
+constexpr int kBatch = 4;         // staged records per thread per step of a pass
 
 __device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_t digit) {
   if (valid) atomicAdd(&hist[digit], 1u);
@@ -283,12 +284,19 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   // ---- counting path
   bool done = false;
   if (staged && m > 0) {
+    // every pass over the staged records takes kBatch of them per thread at a
+    // time, loads first, so that their shared-memory latencies overlap
     uint64_t lo = ~0ull, hi = 0ull;
-    for (int i = tid; i < n_st; i += NT) {
-      const uint64_t r = s_rec[i];
-      if (r != 0ull) {
-        lo = r < lo ? r : lo;
-        hi = r > hi ? r : hi;
+    for (int base = tid; base < n_st; base += kBatch * NT) {
+      uint64_t r[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (r[j] != 0ull) {
+          lo = r[j] < lo ? r[j] : lo;
+          hi = r[j] > hi ? r[j] : hi;
+        }
       }
     }
 #pragma unroll
@@ -317,9 +325,13 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       if (lin) return min(2047u, static_cast<uint32_t>((record_score(r) - smin) * scale));
       return static_cast<uint32_t>((r - rlo) >> shift);
     };
-    for (int i = tid; i < n_st; i += NT) {
-      const uint64_t r = s_rec[i];
-      if (r != 0ull) atomicAdd(&s_hist[digit(r)], 1u);
+    for (int base = tid; base < n_st; base += kBatch * NT) {
+      uint64_t r[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j)
+        if (r[j] != 0ull) atomicAdd(&s_hist[digit(r[j])], 1u);
     }
     __syncthreads();
     // descending exclusive scan: thread t owns buckets 2047-8t down to 2040-8t
@@ -368,22 +380,40 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     __syncthreads();
     const int nw = above + cntB;  // records in bucket B and above
     if (nw <= kWinCap && s_maxc <= kRankMax) {
-      for (int i = tid; i < n_st; i += NT) {
-        const uint64_t r = s_rec[i];
-        if (r == 0ull) continue;
-        const uint32_t d = digit(r);
-        if (static_cast<int>(d) >= B) s_win[atomicAdd(&s_cur[d], 1u)] = r;
+      for (int base = tid; base < n_st; base += kBatch * NT) {
+        uint64_t r[kBatch];
+        uint32_t pos[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const uint32_t d = r[j] != 0ull ? digit(r[j]) : 0u;
+          pos[j] = (r[j] != 0ull && static_cast<int>(d) >= B) ? atomicAdd(&s_cur[d], 1u) : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+          if (pos[j] != 0xFFFFFFFFu) s_win[pos[j]] = r[j];
       }
       __syncthreads();
       // s_cur[d] is now the end of bucket d; rank each record inside its
       // bucket and place the winners in order in the (now free) staging buffer
-      for (int i = tid; i < nw; i += NT) {
-        const uint64_t r = s_win[i];
-        const uint32_t d = digit(r);
-        const int end = static_cast<int>(s_cur[d]), beg = end - static_cast<int>(s_hist[d]);
-        int rank = 0;
-        for (int j = beg; j < end; ++j) rank += (s_win[j] > r) ? 1 : 0;
-        if (beg + rank < m) s_rec[beg + rank] = r;
+      for (int base = tid; base < nw; base += kBatch * NT) {
+        uint64_t r[kBatch];
+        int beg[kBatch], end[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < nw ? s_win[base + j * NT] : 0ull;
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const uint32_t d = r[j] != 0ull ? digit(r[j]) : 0u;
+          end[j] = static_cast<int>(s_cur[d]);
+          beg[j] = r[j] != 0ull ? end[j] - static_cast<int>(s_hist[d]) : end[j];
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          int rank = 0;
+          for (int x = beg[j]; x < end[j]; ++x) rank += (s_win[x] > r[j]) ? 1 : 0;
+          if (r[j] != 0ull && beg[j] + rank < m) s_rec[beg[j] + rank] = r[j];
+        }
       }
       __syncthreads();
       for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_rec[i] : 0ull);

@@ -68,6 +68,15 @@ def test_prefill_compaction_long_rows():
     check_prefill(xh, 300, label="long rows H32")
 
 
+@pytest.mark.parametrize("wl", ["causal_16k_h64", "chunk_128k_h32"])
+def test_prefill_two_warpgroup_epilogue(wl):
+    # many keys per selected record (70k keys per row split over CTAs, topk 6):
+    # the launch takes the two-warpgroup epilogue with the head weights in
+    # registers, where short rows take the four-warpgroup one
+    x = make_prefill(wl, T_q=24, T_k=70024, q_offset=70000, seed=81)
+    check_prefill(x, 6, label=f"two warpgroups {wl}")
+
+
 def test_prefill_key_splits_for_few_rows():
     # 8 query rows against 40k keys: few groups, so each group's keys are
     # split across CTAs and merged by the final selection
