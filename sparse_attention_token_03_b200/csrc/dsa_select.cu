@@ -248,10 +248,13 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   const int n_st = staged ? s_staged : 0;
 
   if (staged && n > 0) {
-    volatile int never = 0;
-    mbar_wait(smem_u32(&s_bar), 0, &never, p.err);
-    __syncwarp();
-    if (wid == 0) {  // blank the padding slot after each odd-sized segment
+    // warp 0 alone waits for the copies (the other warps park at the barrier
+    // below instead of spinning on the mbarrier) and blanks the padding slot
+    // after each odd-sized segment
+    if (wid == 0) {
+      volatile int never = 0;
+      mbar_wait(smem_u32(&s_bar), 0, &never, p.err);
+      __syncwarp();
       int off = 0;
       for (int base = 0; base < n_seg; base += 32) {
         int c = 0;
@@ -285,42 +288,67 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   bool done = false;
   if (staged && m > 0) {
     // every pass over the staged records takes kBatch of them per thread at a
-    // time, loads first, so that their shared-memory latencies overlap
-    uint64_t lo = ~0ull, hi = 0ull;
+    // time, loads first, so that their shared-memory latencies overlap.
+    // First the row's smallest and largest score code (the high words;
+    // padding slots are 0 and wrap to the top under c - 1)
+    const uint32_t* s_code = reinterpret_cast<const uint32_t*>(s_rec);
+    uint32_t clo = 0xFFFFFFFFu, chi = 0u;
     for (int base = tid; base < n_st; base += kBatch * NT) {
-      uint64_t r[kBatch];
+      uint32_t c[kBatch];
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
+      for (int j = 0; j < kBatch; ++j) c[j] = base + j * NT < n_st ? s_code[2 * (base + j * NT) + 1] : 0u;
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        if (r[j] != 0ull) {
-          lo = r[j] < lo ? r[j] : lo;
-          hi = r[j] > hi ? r[j] : hi;
-        }
+        clo = min(clo, c[j] - 1u);
+        chi = max(chi, c[j]);
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
-      lo = l2 < lo ? l2 : lo;
-      hi = h2 > hi ? h2 : hi;
-    }
+    clo = __reduce_min_sync(0xFFFFFFFFu, clo);
+    chi = __reduce_max_sync(0xFFFFFFFFu, chi);
     for (int i = tid; i < 2048; i += NT) s_hist[i] = 0u;
     if (lane == 0) {
-      atomicMin(&s_lo, static_cast<unsigned long long>(lo));
-      atomicMax(&s_hi, static_cast<unsigned long long>(hi));
+      atomicMin(&s_lo, static_cast<unsigned long long>(clo + 1u) << 32);
+      atomicMax(&s_hi, (static_cast<unsigned long long>(chi) << 32) | 0xFFFFFFFFull);
     }
     __syncthreads();
     // bucket of a record: linear in its score between the row's smallest and
     // largest score (any digit that never decreases along the record order
     // works; a linear one spreads the winners evenly), or, when that range is
     // zero or not finite, the top 11 bits of (record - smallest record)
+    const float smin = record_score(s_lo), srange = record_score(s_hi) - smin;
+    const float scale = 2047.0f / srange;
+    const bool lin = srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f;
+    if (!lin) {
+      // equal (or non-finite) extreme scores: the exact record range instead
+      uint64_t lo = ~0ull, hi = 0ull;
+      for (int i = tid; i < n_st; i += NT) {
+        const uint64_t r = s_rec[i];
+        if (r != 0ull) {
+          lo = r < lo ? r : lo;
+          hi = r > hi ? r : hi;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        s_lo = ~0ull;
+        s_hi = 0ull;
+      }
+      __syncthreads();
+      if (lane == 0) {
+        atomicMin(&s_lo, static_cast<unsigned long long>(lo));
+        atomicMax(&s_hi, static_cast<unsigned long long>(hi));
+      }
+      __syncthreads();
+    }
     const uint64_t rlo = s_lo;
     const uint64_t span = s_hi - rlo;
     const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 11);  // span >> shift < 2048
-    const float smin = record_score(rlo), srange = record_score(s_hi) - smin;
-    const float scale = 2047.0f / srange;
-    const bool lin = srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f;
     auto digit = [&](uint64_t r) {
       if (lin) return min(2047u, static_cast<uint32_t>((record_score(r) - smin) * scale));
       return static_cast<uint32_t>((r - rlo) >> shift);
@@ -408,12 +436,21 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
           end[j] = static_cast<int>(s_cur[d]);
           beg[j] = r[j] != 0ull ? end[j] - static_cast<int>(s_hist[d]) : end[j];
         }
+        // the batch's bucket scans advance together (independent loads)
+        int rank[kBatch], len = 0;
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
-          int rank = 0;
-          for (int x = beg[j]; x < end[j]; ++x) rank += (s_win[x] > r[j]) ? 1 : 0;
-          if (r[j] != 0ull && beg[j] + rank < m) s_rec[beg[j] + rank] = r[j];
+          rank[j] = 0;
+          len = max(len, end[j] - beg[j]);
         }
+        for (int x = 0; x < len; ++x) {
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j)
+            if (beg[j] + x < end[j]) rank[j] += (s_win[beg[j] + x] > r[j]) ? 1 : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+          if (r[j] != 0ull && beg[j] + rank[j] < m) s_rec[beg[j] + rank[j]] = r[j];
       }
       __syncthreads();
       for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_rec[i] : 0ull);
@@ -430,7 +467,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     int pbits = 0, above = 0;
     if (staged) {
       // start the digits at the highest bit in which the records differ
-      // (s_lo / s_hi were reduced by the counting path)
+      // (s_lo / s_hi bracket the records; the counting path reduced them)
       const uint64_t diff = s_lo ^ s_hi;  // non-zero: records are distinct
       pbits = __clzll(static_cast<long long>(diff));
       prefix = pbits > 0 ? (s_hi >> (64 - pbits)) : 0ull;
