@@ -310,6 +310,15 @@ __host__ __device__ __forceinline__ float code_score(uint32_t c) {
 #endif
 }
 
+// The lowest fp32 score whose record can reach the threshold record thr:
+// the value of thr's score code (-inf for codes at or below the code of
+// -inf).  A finite score below it has a smaller code and so a smaller record;
+// for codes above that of +inf the result is NaN and no score passes.
+__device__ __forceinline__ float threshold_floor(uint64_t thr) {
+  const uint32_t c = static_cast<uint32_t>(thr >> 32);
+  return c <= 0x007FFFFFu ? -INFINITY : code_score(c);
+}
+
 // Record = (score code << 32) | (0xFFFFFFFF - key).  Ordering records as
 // unsigned 64-bit integers is the selection order: score descending, then
 // key ascending.  Keys are < 2^31, so a record is never 0.

@@ -610,6 +610,23 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         rlo[i] = 0xFFFFFFFFu;
         rhi[i] = 0u;
       }
+      // per query: the admission threshold (record, and the lowest fp32 score
+      // that can reach it) and this warp's append region in the active half.
+      // They change only in the periodic check below, which reloads them.
+      uint64_t thr[GQ];
+      float thr_f[GQ];
+      uint64_t* app[GQ];
+      auto reload = [&]() {
+#pragma unroll
+        for (int i = 0; i < GQ; ++i) {
+          const int qq = q_lo + i;
+          thr[i] = s_thr[qq];
+          thr_f[i] = threshold_floor(thr[i]);
+          app[i] = cand_unit + static_cast<size_t>(qq) * lay.query_recs() +
+                   static_cast<size_t>(s_half[qq]) * lay.half_recs() + lay.region_off(1 + quarter);
+        }
+      };
+      reload();
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
         if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
@@ -619,13 +636,6 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
         if (p.mode == kModeRefine && key_local < U.vis_base)
           key_id = static_cast<uint32_t>(p.surv_ids[U.row0 * p.surv_stride + key_local]);
-        uint64_t thr[GQ];
-        int half[GQ];
-#pragma unroll
-        for (int i = 0; i < GQ; ++i) {
-          thr[i] = s_thr[q_lo + i];
-          half[i] = s_half[q_lo + i];
-        }
         // this warpgroup's GQ x H dot products, read in 16-column chunks: the
         // next chunk's TMEM load overlaps the current chunk's head sums
         constexpr int CPQ = H / 16, NC = GQ * CPQ;
@@ -663,22 +673,25 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
-          bool valid = qq < U.rows;
-          if (p.mode == kModePrefill) valid = valid && key_local < U.vis_base + qq;
-          else valid = valid && key_local < U.vis_base;
-          const uint64_t rec = make_record(score[i], key_id);
-          const bool admit = valid && rec >= thr[i];
-          const uint32_t bal = __ballot_sync(0xFFFFFFFFu, admit);
-          if (admit) {
-            uint64_t* reg = cand_unit + static_cast<size_t>(qq) * lay.query_recs() +
-                            static_cast<size_t>(half[i]) * lay.half_recs() + lay.region_off(1 + quarter);
-            reg[cnt[i] + __popc(bal & lt_mask)] = rec;
-            const uint32_t code = static_cast<uint32_t>(rec >> 32);
-            atomicAdd(&s_qh[qq * kHistBins + (code >> kHistShift)], 1u);
-            rlo[i] = min(rlo[i], code);
-            rhi[i] = max(rhi[i], code);
+          // keys of this tile visible to the query: local keys below lim
+          const int64_t lim64 = (p.mode == kModePrefill ? U.vis_base + qq : U.vis_base) - t * kTileKeys;
+          const int lim = lim64 < 0 ? 0 : (lim64 > kTileKeys ? kTileKeys : static_cast<int>(lim64));
+          // one float compare rules out keys that cannot reach the threshold;
+          // the exact record test runs only in warps where some lane passes
+          const bool pre = qq < U.rows && row_in_tile < lim && score[i] >= thr_f[i];
+          if (__any_sync(0xFFFFFFFFu, pre)) {
+            const uint64_t rec = make_record(score[i], key_id);
+            const bool admit = pre && rec >= thr[i];
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, admit);
+            if (admit) {
+              app[i][cnt[i] + __popc(bal & lt_mask)] = rec;
+              const uint32_t code = static_cast<uint32_t>(rec >> 32);
+              atomicAdd(&s_qh[qq * kHistBins + (code >> kHistShift)], 1u);
+              rlo[i] = min(rlo[i], code);
+              rhi[i] = max(rhi[i], code);
+            }
+            cnt[i] += __popc(bal);
           }
-          cnt[i] += __popc(bal);
         }
         // every kCheckTiles-th tile (and at the unit's end) the warpgroup
         // publishes its append counts, raises each row's admission threshold
@@ -796,6 +809,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           rlo[i] = 0xFFFFFFFFu;
           epi_sync(bar);
         }
+        reload();
       }
       if (!ok) break;
       epi_sync(bar);
