@@ -43,10 +43,35 @@ constexpr int kSelectThreads = 256;
 constexpr int kWideKeysPerRecord = 256;
 
 constexpr int kMetaInts = 8;
-// Score-code histogram of a query's buffered records: bin = code >> 22
-// (sign, exponent and one mantissa bit of the fp32 score: half-octave bins).
+// Score-code histogram of a query's buffered records, 1024 bins: 1/8-octave
+// bins (a score's exponent and top three mantissa bits) over positive scores
+// in [2^-32, 2^32) are bins 512 .. 1023, the mirror image over negative scores
+// in (-2^32, -2^-32] bins 0 .. 511; smaller magnitudes go to bin 511 or 512
+// and larger ones to bins 0 and 1023.  The bin never decreases along the
+// score order, and hist_edge(b) is the smallest score code in bin b.  Signed
+// bins keep the admissions of a row's first keys (threshold still at its
+// minimum, scores of both signs) spread over many bins.
 constexpr int kHistBins = 1024;
-constexpr int kHistShift = 22;
+constexpr uint32_t kHistFine0 = 768u;  // (exponent << 3 | 3 mantissa bits) of 2^-32
+__host__ __device__ constexpr uint32_t hist_clamp511(uint32_t fine) {
+  return fine < kHistFine0 ? 0u : (fine - kHistFine0 > 511u ? 511u : fine - kHistFine0);
+}
+__host__ __device__ constexpr uint32_t hist_bin(uint32_t code) {
+  return (code & 0x80000000u) ? 512u + hist_clamp511((code & 0x7FFFFFFFu) >> 20)
+                              : 511u - hist_clamp511((~code & 0x7FFFFFFFu) >> 20);
+}
+__host__ __device__ constexpr uint32_t hist_edge(uint32_t bin) {
+  return bin >= 513u ? (0x80000000u | ((bin - 512u + kHistFine0) << 20))
+         : bin == 512u ? 0x80000000u
+         : bin == 0u   ? 0u
+                       : 0x7FFFFFFFu - (((kHistFine0 + 511u - bin) << 20) | 0xFFFFFu);
+}
+static_assert(hist_bin(hist_edge(1)) == 1 && hist_bin(hist_edge(1) - 1) == 0 &&
+              hist_bin(hist_edge(511)) == 511 && hist_bin(hist_edge(511) - 1) == 510 &&
+              hist_bin(hist_edge(512)) == 512 && hist_bin(hist_edge(512) - 1) == 511 &&
+              hist_bin(hist_edge(513)) == 513 && hist_bin(hist_edge(513) - 1) == 512 &&
+              hist_bin(hist_edge(1023)) == 1023 && hist_bin(hist_edge(1023) - 1) == 1022,
+              "histogram bins");
 // The epilogue publishes append counts and checks for overflow every
 // kCheckTiles tiles; a warp appends at most 32 records per query per tile.
 constexpr int kCheckTiles = 8;

@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
             if (admit) {
               app[i][cnt[i] + __popc(bal & lt_mask)] = rec;
               const uint32_t code = static_cast<uint32_t>(rec >> 32);
-              atomicAdd(&s_qh[qq * kHistBins + (code >> kHistShift)], 1u);
+              atomicAdd(&s_qh[qq * kHistBins + hist_bin(code)], 1u);
               rlo[i] = min(rlo[i], code);
               rhi[i] = max(rhi[i], code);
             }
@@ -720,7 +720,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           int kept_above = 0;
           if (total >= p.topk && (full || total - s_upd[qq] >= 256)) {
             epi_find_bucket(qh, kHistBins, 0, p.topk, etid, s_misc + 4, s_misc + 1, bar);
-            const uint64_t t_new = static_cast<uint64_t>(static_cast<uint32_t>(s_misc[1]) << kHistShift) << 32;
+            const uint64_t t_new = static_cast<uint64_t>(hist_edge(static_cast<uint32_t>(s_misc[1]))) << 32;
             kept_above = s_misc[2] + s_misc[3];
             epi_sync(bar);
             if (etid == 0) {
@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
             }
             epi_sync(bar);
             // records below the threshold are gone: clear their bins
-            const uint32_t b_thr = static_cast<uint32_t>(thr_q >> (32 + kHistShift));
+            const uint32_t b_thr = hist_bin(static_cast<uint32_t>(thr_q >> 32));
             for (int bb = etid; bb < kHistBins; bb += kEpiThreads)
               if (static_cast<uint32_t>(bb) < b_thr) qh[bb] = 0u;
             if (etid == 0) {
@@ -800,7 +800,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
             const uint64_t* kept = qbuf + static_cast<size_t>(s_half[qq]) * lay.half_recs();
             const int nk = s_count[qq];
             for (int idx = etid; idx < nk; idx += kEpiThreads)
-              atomicAdd(&qh[static_cast<uint32_t>(kept[idx] >> 32) >> kHistShift], 1u);
+              atomicAdd(&qh[hist_bin(static_cast<uint32_t>(kept[idx] >> 32))], 1u);
             epi_sync(bar);
             rhi[i] = static_cast<uint32_t>(hi >> 32);
           }
