@@ -87,6 +87,30 @@ DSA_API int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t*
                       float* out_score, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * The same chunked causal prefill from HOST buffers: q, w and k are host
+ * arrays with the layouts above, out_idx / out_score host arrays
+ * [T_q][topk].  The call copies the keys to the device once and streams the
+ * query rows through in up to 16 row blocks (rows are independent, "DeepSeek
+ * DSA FLOPs", index score): while one block is scored on `stream`, the next
+ * block's inputs and the previous block's outputs cross PCIe on two library
+ * streams, so the copies in both directions overlap the kernels.  Results
+ * equal dsa_index_prefill's bit for bit.  The call is asynchronous: the host
+ * outputs are complete once `stream` has been synchronised.  Host buffers
+ * should be page-locked (cudaHostAlloc / pinned) for the copies to overlap;
+ * pageable buffers work but serialise.  The workspace (device, 256-byte
+ * aligned, dsa_index_prefill_host_workspace_bytes()) holds the prefill
+ * workspace at offset 0 (dsa_index_device_status reads it there), the keys
+ * and two slots of row-block buffers.  Calls are serialised by a library
+ * mutex; the library's two copy streams per device live until the process
+ * exits.  The pages have no counterpart: this is the boundary's host-buffer
+ * form of dsa_index_prefill.
+ */
+DSA_API size_t dsa_index_prefill_host_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk);
+DSA_API int dsa_index_prefill_host(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                                   int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
+                                   float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Batched decode ("DeepSeek DSA FLOPs", Decode): sequence b has one new query
  * q[b] (H rows) and its own key cache k_cache[b] of capacity t_cap, of which
  * the first seq_len[b] keys are visible (the new token's key included).

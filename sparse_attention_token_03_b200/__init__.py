@@ -21,6 +21,7 @@ __all__ = [
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
     "dsa_index_decode_noalloc", "dsa_index_prefill_pruned", "dsa_index_prefill_pruned_workspace_bytes",
+    "dsa_index_prefill_host", "dsa_index_prefill_host_workspace_bytes",
 ]
 
 DSA_OK = 0
@@ -55,6 +56,10 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_prefill_workspace_bytes.restype = SZ
         L.dsa_index_prefill.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
         L.dsa_index_prefill.restype = I
+        L.dsa_index_prefill_host_workspace_bytes.argtypes = [I64, I64, I, I, I]
+        L.dsa_index_prefill_host_workspace_bytes.restype = SZ
+        L.dsa_index_prefill_host.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_prefill_host.restype = I
         L.dsa_index_decode_workspace_bytes.argtypes = [I, I64, I, I, I]
         L.dsa_index_decode_workspace_bytes.restype = SZ
         L.dsa_index_decode.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]
@@ -148,6 +153,56 @@ def dsa_index_prefill(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offse
                                        T_k, H, d, int(topk), out_idx.data_ptr(),
                                        out_score.data_ptr(), ws.data_ptr(), ws.numel(),
                                        _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_prefill_host_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int) -> int:
+    return int(lib().dsa_index_prefill_host_workspace_bytes(T_q, T_k, H, d, topk))
+
+
+def _need_host(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.dim() != ndim:
+        raise TypeError(f"{name} must be a {ndim}-dim {dtype} tensor, got {t.dtype} {tuple(t.shape)}")
+    if t.device.type != "cpu" or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host (CPU) tensor")
+
+
+def dsa_index_prefill_host(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offset: int, topk: int,
+                           out_idx=None, out_score=None, workspace=None, device=None):
+    """dsa_index_prefill from host buffers, with the copies pipelined.
+
+    q (T_q, H, d) bf16, w (T_q, H) fp32, k (T_k, d) bf16 are CPU tensors
+    (page-locked ones let the copies overlap the kernels); the outputs are
+    CPU tensors (T_q, topk) (page-locked ones are allocated when not given).
+    The work is queued on the current stream of ``device`` (default: the
+    current CUDA device); the outputs are complete after that stream is
+    synchronised.
+    """
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _need_host(q, "q", torch.bfloat16, 3)
+    _need_host(w, "w", torch.float32, 2)
+    _need_host(k, "k", torch.bfloat16, 2)
+    T_q, H, d = q.shape
+    T_k = k.shape[0]
+    if tuple(w.shape) != (T_q, H) or k.shape[1] != d:
+        raise ValueError("shape mismatch between q (T_q,H,d), w (T_q,H) and k (T_k,d)")
+    if out_idx is None:
+        out_idx = torch.empty((T_q, topk), dtype=torch.int32).pin_memory()
+    if out_score is None:
+        out_score = torch.empty((T_q, topk), dtype=torch.float32).pin_memory()
+    _need_host(out_idx, "out_idx", torch.int32, 2)
+    _need_host(out_score, "out_score", torch.float32, 2)
+    if tuple(out_idx.shape) != (T_q, topk) or tuple(out_score.shape) != (T_q, topk):
+        raise ValueError(f"outputs must be ({T_q}, {topk})")
+    nbytes = dsa_index_prefill_host_workspace_bytes(T_q, T_k, H, d, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_host(q.data_ptr(), w.data_ptr(), k.data_ptr(), int(q_offset), T_q,
+                                            T_k, H, d, int(topk), out_idx.data_ptr(),
+                                            out_score.data_ptr(), ws.data_ptr(), ws.numel(),
+                                            _stream_ptr(dev)))
     return out_idx, out_score
 
 

@@ -367,45 +367,29 @@ int noalloc_scratch(void** out) {
   return DSA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* dsa_last_error_string(void) { return g_last_error.c_str(); }
-
-size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
-  if (check_shape(H, d, topk) != DSA_OK || T_q < 0 || T_k < 1) return 0;
-  // the split choice depends on q_offset; size for the most splits (q_offset = T_k - T_q)
-  return plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
-}
-
-int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
-                      int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
-                      float* out_score, void* workspace, size_t ws_bytes, void* stream) {
+int check_prefill_args(int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d, int topk) {
   int rc = check_shape(H, d, topk);
   if (rc != DSA_OK) return rc;
   if (T_q < 0 || T_k < 1 || q_offset < 0 || q_offset + T_q > T_k)
     return fail(DSA_EINVAL, "need T_q >= 0, T_k >= 1, 0 <= q_offset, q_offset + T_q <= T_k");
   if (T_k >= (int64_t(1) << 31) || T_q * H >= (int64_t(1) << 31))
     return fail(DSA_EINVAL, "T_k and T_q*H must be below 2^31");
-  if (T_q == 0) return DSA_OK;
-  if (!q || !w || !k || !out_idx || !out_score || !workspace)
-    return fail(DSA_EINVAL, "null pointer argument");
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
-      !aligned(out_idx, 4) || !aligned(out_score, 4))
-    return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
-  const PrefillPlan P = plan_prefill(T_q, T_k, q_offset, H, topk);
-  const size_t need = plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
-  if (ws_bytes < std::max(need, P.bytes))
-    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, std::max(need, P.bytes));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return DSA_OK;
+}
+
+// Fused score + streaming Top-k over the chunk's rows, then the final
+// selection, on device buffers (arguments already checked).  reset_status
+// clears the workspace's device status word first.
+int prefill_run(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset, int64_t T_q,
+                int64_t T_k, int H, int topk, int32_t* out_idx, float* out_score, uint8_t* ws,
+                const PrefillPlan& P, bool reset_status, bool profile, cudaStream_t st) {
+  int rc;
   CUtensorMap tq, tk;
   if ((rc = make_tmap(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
   if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
-  cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  prof_begin(st);
+  cudaError_t e;
+  if (reset_status && (e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (profile) prof_begin(st);
 
   ScoreParams sp{};
   sp.mode = kModePrefill;
@@ -422,7 +406,7 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = reinterpret_cast<uint32_t*>(ws);
   if ((e = launch_score(H, P.G, P.eg, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
-  prof_mark(st, "score_topk");
+  if (profile) prof_mark(st, "score_topk");
 
   SelectParams se{};
   se.mode = kModePrefill;
@@ -437,8 +421,175 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   se.out_score = out_score;
   se.err = sp.err;
   if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
-  prof_mark(st, "select_topk");
+  if (profile) prof_mark(st, "select_topk");
   return DSA_OK;
+}
+
+// ------------------------------------------------------- host-buffer prefill
+// Row blocks of a chunk stream through two device slots: while block b is
+// scored on the caller's stream, the inputs of block b+1 cross PCIe on one
+// library stream and the outputs of block b-1 come back on another (the two
+// copy directions run at once).  Keys go to the device once per call.
+struct HostPlan {
+  int64_t block_rows;
+  int nb;
+  size_t off_k, off_q[2], off_w[2], off_idx[2], off_score[2], off_ws, ws_bytes, bytes;
+};
+
+HostPlan plan_host(int64_t T_q, int64_t T_k, int H, int d, int topk) {
+  HostPlan P{};
+  const int64_t nb = std::min<int64_t>(std::max<int64_t>((T_q + 2047) / 2048, 1), 16);
+  P.block_rows = std::max<int64_t>(((T_q + nb - 1) / nb + 7) / 8 * 8, 1);
+  P.nb = static_cast<int>((T_q + P.block_rows - 1) / P.block_rows);
+  const int64_t br = P.block_rows, last = T_q - (P.nb - 1) * br;
+  // one prefill workspace first (its device status word at offset 0, where
+  // dsa_index_device_status reads it), reused block after block on the
+  // caller's stream; then the keys and two slots of block buffers
+  P.ws_bytes = std::max(plan_prefill(br, T_k, T_k - br, H, topk).bytes,
+                        plan_prefill(last, T_k, T_k - last, H, topk).bytes);
+  P.off_ws = 0;
+  size_t off = align_up(P.ws_bytes, 256);
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = align_up(off + n, 256);
+    return o;
+  };
+  P.off_k = take(static_cast<size_t>(T_k) * d * 2);
+  for (int s = 0; s < 2; ++s) {
+    P.off_q[s] = take(static_cast<size_t>(br) * H * d * 2);
+    P.off_w[s] = take(static_cast<size_t>(br) * H * 4);
+    P.off_idx[s] = take(static_cast<size_t>(br) * topk * 4);
+    P.off_score[s] = take(static_cast<size_t>(br) * topk * 4);
+  }
+  P.bytes = off;
+  return P;
+}
+
+struct HostStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, keys = nullptr;
+  cudaEvent_t in[16] = {}, comp[16] = {}, out[16] = {};
+};
+
+std::mutex g_host_mu;
+
+int host_streams(HostStreams** out) {
+  static HostStreams per_dev[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(DSA_EDEVICE, "device ordinal %d out of range", dev);
+  HostStreams& H = per_dev[dev];
+  if (!H.h2d) {
+    auto ev = [&](cudaEvent_t* x) { return cudaEventCreateWithFlags(x, cudaEventDisableTiming); };
+    if ((e = cudaStreamCreateWithFlags(&H.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&H.d2h, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = ev(&H.start)) != cudaSuccess || (e = ev(&H.keys)) != cudaSuccess)
+      return cuda_fail(e, "library stream/event creation");
+    for (int i = 0; i < 16; ++i)
+      if ((e = ev(&H.in[i])) != cudaSuccess || (e = ev(&H.comp[i])) != cudaSuccess ||
+          (e = ev(&H.out[i])) != cudaSuccess)
+        return cuda_fail(e, "library event creation");
+  }
+  *out = &H;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_last_error_string(void) { return g_last_error.c_str(); }
+
+size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
+  if (check_shape(H, d, topk) != DSA_OK || T_q < 0 || T_k < 1) return 0;
+  // the split choice depends on q_offset; size for the most splits (q_offset = T_k - T_q)
+  return plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
+}
+
+int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                      int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
+                      float* out_score, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_prefill_args(q_offset, T_q, T_k, H, d, topk);
+  if (rc != DSA_OK || T_q == 0) return rc;
+  if (!q || !w || !k || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
+  const size_t need = dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk);
+  const PrefillPlan P = plan_prefill(T_q, T_k, q_offset, H, topk);
+  if (ws_bytes < std::max(need, P.bytes))
+    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, std::max(need, P.bytes));
+  return prefill_run(q, w, k, q_offset, T_q, T_k, H, topk, out_idx, out_score,
+                     static_cast<uint8_t*>(workspace), P, true, true, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_index_prefill_host_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
+  if (check_shape(H, d, topk) != DSA_OK || T_q < 1 || T_k < 1) return 0;
+  return plan_host(T_q, T_k, H, d, topk).bytes;
+}
+
+int dsa_index_prefill_host(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
+                           int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
+                           float* out_score, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_prefill_args(q_offset, T_q, T_k, H, d, topk);
+  if (rc != DSA_OK || T_q == 0) return rc;
+  if (!q || !w || !k || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(workspace, 256)) return fail(DSA_EINVAL, "misaligned workspace (needs 256 bytes)");
+  const HostPlan P = plan_host(T_q, T_k, H, d, topk);
+  if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostStreams* S = nullptr;
+  if ((rc = host_streams(&S)) != DSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* pws = ws + P.off_ws;
+  auto ck = [&](cudaError_t x, const char* what) { return x == cudaSuccess ? DSA_OK : cuda_fail(x, what); };
+  // the copy streams start after everything already queued on the caller's stream
+  if ((rc = ck(cudaEventRecord(S->start, st), "cudaEventRecord")) != DSA_OK) return rc;
+  if ((rc = ck(cudaStreamWaitEvent(S->h2d, S->start, 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+  if ((rc = ck(cudaStreamWaitEvent(S->d2h, S->start, 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+  if ((rc = ck(cudaMemsetAsync(pws, 0, 4, st), "cudaMemsetAsync")) != DSA_OK) return rc;
+  uint16_t* dk = reinterpret_cast<uint16_t*>(ws + P.off_k);
+  if ((rc = ck(cudaMemcpyAsync(dk, k, static_cast<size_t>(T_k) * d * 2, cudaMemcpyHostToDevice, S->h2d),
+               "key copy")) != DSA_OK) return rc;
+  if ((rc = ck(cudaEventRecord(S->keys, S->h2d), "cudaEventRecord")) != DSA_OK) return rc;
+  if ((rc = ck(cudaStreamWaitEvent(st, S->keys, 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+  for (int b = 0; b < P.nb; ++b) {
+    const int s = b & 1;
+    const int64_t r0 = b * P.block_rows, rows = std::min(P.block_rows, T_q - r0);
+    uint16_t* dq = reinterpret_cast<uint16_t*>(ws + P.off_q[s]);
+    float* dw = reinterpret_cast<float*>(ws + P.off_w[s]);
+    int32_t* di = reinterpret_cast<int32_t*>(ws + P.off_idx[s]);
+    float* dsc = reinterpret_cast<float*>(ws + P.off_score[s]);
+    // inputs of block b, once slot s is free (block b-2's outputs copied out)
+    if (b >= 2 && (rc = ck(cudaStreamWaitEvent(S->h2d, S->out[b - 2], 0), "cudaStreamWaitEvent")) != DSA_OK)
+      return rc;
+    if ((rc = ck(cudaMemcpyAsync(dq, q + r0 * H * d, static_cast<size_t>(rows) * H * d * 2,
+                                 cudaMemcpyHostToDevice, S->h2d), "query copy")) != DSA_OK) return rc;
+    if ((rc = ck(cudaMemcpyAsync(dw, w + r0 * H, static_cast<size_t>(rows) * H * 4, cudaMemcpyHostToDevice,
+                                 S->h2d), "weight copy")) != DSA_OK) return rc;
+    if ((rc = ck(cudaEventRecord(S->in[b], S->h2d), "cudaEventRecord")) != DSA_OK) return rc;
+    // score block b on the caller's stream
+    if ((rc = ck(cudaStreamWaitEvent(st, S->in[b], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+    const PrefillPlan PB = plan_prefill(rows, T_k, q_offset + r0, H, topk);
+    if (PB.bytes > P.ws_bytes) return fail(DSA_EWORKSPACE, "internal: block workspace too small");
+    if ((rc = prefill_run(dq, dw, dk, q_offset + r0, rows, T_k, H, topk, di, dsc, pws, PB, false, false, st)) !=
+        DSA_OK)
+      return rc;
+    if ((rc = ck(cudaEventRecord(S->comp[b], st), "cudaEventRecord")) != DSA_OK) return rc;
+    // its outputs back to the host
+    if ((rc = ck(cudaStreamWaitEvent(S->d2h, S->comp[b], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+    if ((rc = ck(cudaMemcpyAsync(out_idx + r0 * topk, di, static_cast<size_t>(rows) * topk * 4,
+                                 cudaMemcpyDeviceToHost, S->d2h), "index copy")) != DSA_OK) return rc;
+    if ((rc = ck(cudaMemcpyAsync(out_score + r0 * topk, dsc, static_cast<size_t>(rows) * topk * 4,
+                                 cudaMemcpyDeviceToHost, S->d2h), "score copy")) != DSA_OK) return rc;
+    if ((rc = ck(cudaEventRecord(S->out[b], S->d2h), "cudaEventRecord")) != DSA_OK) return rc;
+  }
+  // the caller's stream completes when the last outputs are on the host
+  return ck(cudaStreamWaitEvent(st, S->out[P.nb - 1], 0), "cudaStreamWaitEvent");
 }
 
 size_t dsa_index_decode_workspace_bytes(int B, int64_t t_cap, int H, int d, int topk) {

@@ -77,6 +77,41 @@ def test_prefill_two_warpgroup_epilogue(wl):
     check_prefill(x, 6, label=f"two warpgroups {wl}")
 
 
+def _host(a, dtype, pinned):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    t = t.view(torch.int16).view(torch.bfloat16) if dtype == torch.bfloat16 else t
+    return t.pin_memory() if pinned else t
+
+
+@pytest.mark.parametrize("wl,T_q,off,topk,pinned", [("causal_16k_h64", 5000, 100, 256, True),
+                                                    ("chunk_128k_h32", 37, 3000, 64, False),
+                                                    ("causal_16k_h64", 16384, 0, 2048, True)])
+def test_prefill_host_buffers_match_device_call(wl, T_q, off, topk, pinned):
+    # host inputs and outputs, rows streamed in blocks through two device
+    # slots (ragged last block; one block; eight blocks at the benchmark's
+    # size): bit for bit the device call's result, twice in a row
+    x = make_prefill(wl, T_q=T_q, T_k=off + T_q, q_offset=off, seed=900 + T_q)
+    di, ds = run_prefill(x, topk)
+    hq, hw, hk = _host(x["q"].view(np.int16), torch.bfloat16, pinned), _host(x["w"], torch.float32, pinned), \
+        _host(x["k"].view(np.int16), torch.bfloat16, pinned)
+    ws = torch.empty(dsa.dsa_index_prefill_host_workspace_bytes(T_q, off + T_q, x["H"], 128, topk),
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        hi, hs = dsa.dsa_index_prefill_host(hq, hw, hk, off, topk, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(hi.numpy(), di)
+        assert np.array_equal(hs.numpy().view(np.uint32), ds.view(np.uint32))
+    assert dsa.dsa_index_device_status(ws) == 0
+
+
+def test_prefill_host_rejects_device_tensors():
+    x = make_prefill("causal_16k_h64", T_q=8, T_k=8, q_offset=0, seed=3)
+    q = _host(x["q"].view(np.int16), torch.bfloat16, False)
+    with pytest.raises(ValueError):
+        dsa.dsa_index_prefill_host(q.cuda(), _host(x["w"], torch.float32, False),
+                                   _host(x["k"].view(np.int16), torch.bfloat16, False), 0, 4)
+
+
 def test_prefill_key_splits_for_few_rows():
     # 8 query rows against 40k keys: few groups, so each group's keys are
     # split across CTAs and merged by the final selection
