@@ -557,36 +557,39 @@ int dsa_index_prefill_host(const uint16_t* q, const float* w, const uint16_t* k,
                "key copy")) != DSA_OK) return rc;
   if ((rc = ck(cudaEventRecord(S->keys, S->h2d), "cudaEventRecord")) != DSA_OK) return rc;
   if ((rc = ck(cudaStreamWaitEvent(st, S->keys, 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
-  for (int b = 0; b < P.nb; ++b) {
-    const int s = b & 1;
+  // last block first: under a causal mask later rows see more keys, so the
+  // longest scoring overlaps the copies and the exposed tail is short
+  for (int i = 0; i < P.nb; ++i) {
+    const int b = P.nb - 1 - i, s = i & 1;
     const int64_t r0 = b * P.block_rows, rows = std::min(P.block_rows, T_q - r0);
     uint16_t* dq = reinterpret_cast<uint16_t*>(ws + P.off_q[s]);
     float* dw = reinterpret_cast<float*>(ws + P.off_w[s]);
     int32_t* di = reinterpret_cast<int32_t*>(ws + P.off_idx[s]);
     float* dsc = reinterpret_cast<float*>(ws + P.off_score[s]);
-    // inputs of block b, once slot s is free (block b-2's outputs copied out)
-    if (b >= 2 && (rc = ck(cudaStreamWaitEvent(S->h2d, S->out[b - 2], 0), "cudaStreamWaitEvent")) != DSA_OK)
+    // inputs of block b, once slot s is free (the outputs of the block two
+    // steps earlier copied out)
+    if (i >= 2 && (rc = ck(cudaStreamWaitEvent(S->h2d, S->out[i - 2], 0), "cudaStreamWaitEvent")) != DSA_OK)
       return rc;
     if ((rc = ck(cudaMemcpyAsync(dq, q + r0 * H * d, static_cast<size_t>(rows) * H * d * 2,
                                  cudaMemcpyHostToDevice, S->h2d), "query copy")) != DSA_OK) return rc;
     if ((rc = ck(cudaMemcpyAsync(dw, w + r0 * H, static_cast<size_t>(rows) * H * 4, cudaMemcpyHostToDevice,
                                  S->h2d), "weight copy")) != DSA_OK) return rc;
-    if ((rc = ck(cudaEventRecord(S->in[b], S->h2d), "cudaEventRecord")) != DSA_OK) return rc;
+    if ((rc = ck(cudaEventRecord(S->in[i], S->h2d), "cudaEventRecord")) != DSA_OK) return rc;
     // score block b on the caller's stream
-    if ((rc = ck(cudaStreamWaitEvent(st, S->in[b], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+    if ((rc = ck(cudaStreamWaitEvent(st, S->in[i], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
     const PrefillPlan PB = plan_prefill(rows, T_k, q_offset + r0, H, topk);
     if (PB.bytes > P.ws_bytes) return fail(DSA_EWORKSPACE, "internal: block workspace too small");
     if ((rc = prefill_run(dq, dw, dk, q_offset + r0, rows, T_k, H, topk, di, dsc, pws, PB, false, false, st)) !=
         DSA_OK)
       return rc;
-    if ((rc = ck(cudaEventRecord(S->comp[b], st), "cudaEventRecord")) != DSA_OK) return rc;
+    if ((rc = ck(cudaEventRecord(S->comp[i], st), "cudaEventRecord")) != DSA_OK) return rc;
     // its outputs back to the host
-    if ((rc = ck(cudaStreamWaitEvent(S->d2h, S->comp[b], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
+    if ((rc = ck(cudaStreamWaitEvent(S->d2h, S->comp[i], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
     if ((rc = ck(cudaMemcpyAsync(out_idx + r0 * topk, di, static_cast<size_t>(rows) * topk * 4,
                                  cudaMemcpyDeviceToHost, S->d2h), "index copy")) != DSA_OK) return rc;
     if ((rc = ck(cudaMemcpyAsync(out_score + r0 * topk, dsc, static_cast<size_t>(rows) * topk * 4,
                                  cudaMemcpyDeviceToHost, S->d2h), "score copy")) != DSA_OK) return rc;
-    if ((rc = ck(cudaEventRecord(S->out[b], S->d2h), "cudaEventRecord")) != DSA_OK) return rc;
+    if ((rc = ck(cudaEventRecord(S->out[i], S->d2h), "cudaEventRecord")) != DSA_OK) return rc;
   }
   // the caller's stream completes when the last outputs are on the host
   return ck(cudaStreamWaitEvent(st, S->out[P.nb - 1], 0), "cudaStreamWaitEvent");
