@@ -196,6 +196,9 @@ DSA_API int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const ui
  * every device-side check passed.  Synchronises `stream`.
  * Bit 0: a bounded wait inside a kernel gave up (the kernel unwound).
  * Bit 1: a capacity or length check failed.  Bit 2: the seed list was invalid.
+ * Bit 3: a causally visible (query, key) pair scored inf or NaN, i.e. q, k or
+ * w holds a non-finite value; such pairs are never selected and the rows
+ * they belong to are unspecified.
  */
 DSA_API int dsa_index_device_status(const void* workspace, uint32_t* status, void* stream);
 

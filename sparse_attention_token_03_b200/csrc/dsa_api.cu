@@ -854,6 +854,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     stats->records = T_q * static_cast<int64_t>(topk) + static_cast<int64_t>(h[1]);
     if (status & kErrSeed) return fail(DSA_ESEED, "a seed was out of range or repeated; the rows were recomputed densely");
     if (status & kErrTimeout) return fail(DSA_EDEVICE, "a device-side wait gave up (status 0x%x)", status);
+    if (status & kErrNonFinite) return fail(DSA_EDEVICE, "a visible pair scored inf or NaN (non-finite input)");
   }
   return DSA_OK;
 }

@@ -18,6 +18,7 @@ enum : uint32_t {
   kErrTimeout = 1u << 0,   // a bounded wait gave up
   kErrOverflow = 1u << 1,  // a fixed-capacity buffer would have overflowed
   kErrSeed = 1u << 2,      // the seed list failed validation
+  kErrNonFinite = 1u << 3, // a causally visible pair scored inf or NaN (non-finite input)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -627,6 +627,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         }
       };
       reload();
+      bool nonfinite = false;  // a visible pair scored inf or NaN (reported at the unit's end)
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
         if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
@@ -678,7 +679,9 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           const int lim = lim64 < 0 ? 0 : (lim64 > kTileKeys ? kTileKeys : static_cast<int>(lim64));
           // one float compare rules out keys that cannot reach the threshold;
           // the exact record test runs only in warps where some lane passes
-          const bool pre = qq < U.rows && row_in_tile < lim && score[i] >= thr_f[i];
+          const bool vis = qq < U.rows && row_in_tile < lim;
+          nonfinite = nonfinite || (vis && !(fabsf(score[i]) <= 3.402823466e38f));
+          const bool pre = vis && score[i] >= thr_f[i];
           if (__any_sync(0xFFFFFFFFu, pre)) {
             const uint64_t rec = make_record(score[i], key_id);
             const bool admit = pre && rec >= thr[i];
@@ -811,6 +814,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         }
         reload();
       }
+      if (__any_sync(0xFFFFFFFFu, nonfinite) && lane == 0) atomicOr(p.err, kErrNonFinite);
       if (!ok) break;
       epi_sync(bar);
       if (etid < GQ) {

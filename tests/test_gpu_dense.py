@@ -112,6 +112,27 @@ def test_prefill_host_rejects_device_tensors():
                                    _host(x["k"].view(np.int16), torch.bfloat16, False), 0, 4)
 
 
+def test_non_finite_inputs_set_the_status_bit():
+    # a NaN key or an inf query entry inside the causal window sets status
+    # bit 3; a NaN in a key no row can see leaves the status clean
+    def status_after(q, k, off=0):
+        ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(q.shape[0], k.shape[0], 64, 128, 16),
+                         dtype=torch.uint8, device="cuda")
+        dsa.dsa_index_prefill(bf16(q), f32(x["w"]), bf16(k), off, 16, workspace=ws)
+        return dsa.dsa_index_device_status(ws)
+    x = make_prefill("causal_16k_h64", T_q=32, T_k=64, q_offset=0, seed=11)
+    assert status_after(x["q"], x["k"]) == 0
+    k = x["k"].copy()
+    k[10, 5] = 0x7FC0  # bf16 NaN, visible to rows 10..31
+    assert status_after(x["q"], k) & 8
+    q = x["q"].copy()
+    q[3, 7, 0] = 0x7F80  # bf16 +inf in one head of row 3
+    assert status_after(q, x["k"]) & 8
+    k = x["k"].copy()
+    k[50, 0] = 0x7FC0  # past every row's causal window
+    assert status_after(x["q"], k) == 0
+
+
 def test_prefill_key_splits_for_few_rows():
     # 8 query rows against 40k keys: few groups, so each group's keys are
     # split across CTAs and merged by the final selection
