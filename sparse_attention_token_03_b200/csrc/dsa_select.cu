@@ -443,10 +443,13 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
           rank[j] = 0;
           len = max(len, end[j] - beg[j]);
         }
-        for (int x = 0; x < len; ++x) {
+        for (int x = 0; x < len; x += 2) {
 #pragma unroll
-          for (int j = 0; j < kBatch; ++j)
-            if (beg[j] + x < end[j]) rank[j] += (s_win[beg[j] + x] > r[j]) ? 1 : 0;
+          for (int j = 0; j < kBatch; ++j) {
+            const uint64_t a0 = beg[j] + x < end[j] ? s_win[beg[j] + x] : 0ull;
+            const uint64_t a1 = beg[j] + x + 1 < end[j] ? s_win[beg[j] + x + 1] : 0ull;
+            rank[j] += (a0 > r[j] ? 1 : 0) + (a1 > r[j] ? 1 : 0);
+          }
         }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j)
