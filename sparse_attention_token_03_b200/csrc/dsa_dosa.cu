@@ -130,15 +130,37 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
   }
   __syncthreads();
 
-  // importance: NT / H threads per head, each over a fixed slice of samples
+  // importance: NT / H threads per head, each over a fixed slice of samples,
+  // four samples at a time (four independent FMA chains, each over e in
+  // ascending order) reading bf16 pairs
   {
     constexpr int TPH = NT / H;
     const int j = tid % H, slice = tid / H;
+    const uint32_t* qj = reinterpret_cast<const uint32_t*>(&qf[j][0]);
     float acc = 0.0f;
-    for (int s = slice; s < nsamp; s += TPH) {
-      float d = 0.0f;
-      for (int e = 0; e < kD; ++e) d = fmaf(bf16_to_f32(qf[j][e]), bf16_to_f32(kf[s][e]), d);
-      acc += fmaxf(d, 0.0f);
+    for (int s0 = slice; s0 < nsamp; s0 += 4 * TPH) {
+      const uint32_t* ks[4];
+      float d[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int sm = s0 + m * TPH;
+        ks[m] = reinterpret_cast<const uint32_t*>(&kf[sm < nsamp ? sm : 0][0]);
+        d[m] = 0.0f;
+      }
+#pragma unroll 4
+      for (int e2 = 0; e2 < kD / 2; ++e2) {
+        const uint32_t qp = qj[e2];
+        const float q0 = __uint_as_float(qp << 16), q1 = __uint_as_float(qp & 0xFFFF0000u);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t kp = ks[m][e2];
+          d[m] = fmaf(q0, __uint_as_float(kp << 16), d[m]);
+          d[m] = fmaf(q1, __uint_as_float(kp & 0xFFFF0000u), d[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (s0 + m * TPH < nsamp) acc += fmaxf(d[m], 0.0f);
     }
     part[tid] = acc;
     __syncthreads();
@@ -155,17 +177,29 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
     }
     __syncthreads();
   }
-  // retained heads: largest importance first, smaller index on ties
-  if (tid == 0) {
-    unsigned long long taken = 0ull;
+  // retained heads: largest importance first, smaller index on ties (warp 0:
+  // lane l holds heads l and l + 32; importances are >= 0, -1 marks taken)
+  if (wid == 0) {
+    float v0 = lane < H ? imp[lane] : -1.0f, v1 = lane + 32 < H ? imp[lane + 32] : -1.0f;
     for (int a = 0; a < R; ++a) {
-      int best = -1;
-      for (int j = 0; j < H; ++j) {
-        if ((taken >> j) & 1ull) continue;
-        if (best < 0 || imp[j] > imp[best]) best = j;
+      float bv = v0;
+      int bi = lane;
+      if (v1 > v0) {
+        bv = v1;
+        bi = lane + 32;
       }
-      sel[a] = best;
-      taken |= 1ull << best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (lane == 0) sel[a] = bi;
+      if (bi == lane) v0 = -1.0f;
+      if (bi == lane + 32) v1 = -1.0f;
     }
   }
   __syncthreads();
@@ -179,21 +213,30 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
     if (lane == 0) Lc[a][b] = v;
   }
   __syncthreads();
-  if (tid == 0) {
-    int ok = 1;
-    for (int j = 0; j < R && ok; ++j) {
-      double s = Lc[j][j];
-      for (int k2 = 0; k2 < j; ++k2) s -= Lc[j][k2] * Lc[j][k2];
-      if (!(s > 1e-9 * (1.0 + fabs(Lc[j][j])))) { ok = 0; break; }
-      const double ljj = sqrt(s);
-      Lc[j][j] = ljj;
-      for (int i = j + 1; i < R; ++i) {
-        double v = Lc[i][j];
-        for (int k2 = 0; k2 < j; ++k2) v -= Lc[i][k2] * Lc[j][k2];
-        Lc[i][j] = v / ljj;
+  if (wid == 0) {
+    // Cholesky, one column per step: the diagonal from a warp sum, then lane i
+    // (j < i < R) finishes L[i][j]
+    bool ok = true;
+    for (int j = 0; j < R; ++j) {
+      double sq = lane < j ? Lc[j][lane] * Lc[j][lane] : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
+      const double s = Lc[j][j] - sq;
+      if (!(s > 1e-9 * (1.0 + fabs(Lc[j][j])))) {
+        ok = false;
+        break;
       }
+      const double ljj = sqrt(s);
+      if (lane > j && lane < R) {
+        double v = Lc[lane][j];
+        for (int k2 = 0; k2 < j; ++k2) v -= Lc[lane][k2] * Lc[j][k2];
+        Lc[lane][j] = v / ljj;
+      }
+      __syncwarp();
+      if (lane == 0) Lc[j][j] = ljj;
+      __syncwarp();
     }
-    chol_ok = ok;
+    if (lane == 0) chol_ok = ok ? 1 : 0;
   }
   for (int i = tid; i < 4 * R; i += NT) (&wal[0][0])[i] = 0.0f;
   if (tid < 4) wbe[tid] = 0.0f;
@@ -212,23 +255,25 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
       for (int e = lane; e < kD; e += 32) v = fmaf(bf16_to_f32(qf[sel[a]][e]), bf16_to_f32(qf[j][e]), v);
       b[a] = warp_sum(v);
     }
-    if (lane == 0) {
-      double x[R];
-      for (int a = 0; a < R; ++a) x[a] = chol_ok ? static_cast<double>(b[a]) : 0.0;
-      if (chol_ok) {
-        for (int i = 0; i < R; ++i) {
-          double v = x[i];
-          for (int k2 = 0; k2 < i; ++k2) v -= Lc[i][k2] * x[k2];
-          x[i] = v / Lc[i][i];
-        }
-        for (int i = R - 1; i >= 0; --i) {
-          double v = x[i];
-          for (int k2 = i + 1; k2 < R; ++k2) v -= Lc[k2][i] * x[k2];
-          x[i] = v / Lc[i][i];
-        }
+    // G c = b by the two triangular solves, lane a holding entry a: after
+    // entry i is final, the lanes below (forward) / above (backward) update
+    double x = 0.0;
+#pragma unroll
+    for (int a = 0; a < R; ++a)
+      if (lane == a && chol_ok) x = static_cast<double>(b[a]);
+    if (chol_ok) {
+      for (int i = 0; i < R; ++i) {
+        const double xi = __shfl_sync(0xFFFFFFFFu, x, i) / Lc[i][i];
+        if (lane == i) x = xi;
+        if (lane > i && lane < R) x -= Lc[lane][i] * xi;
       }
-      for (int a = 0; a < R; ++a) coef[wid][a] = static_cast<float>(x[a]);
+      for (int i = R - 1; i >= 0; --i) {
+        const double xi = __shfl_sync(0xFFFFFFFFu, x, i) / Lc[i][i];
+        if (lane == i) x = xi;
+        if (lane < i) x -= Lc[i][lane] * xi;
+      }
     }
+    if (lane < R) coef[wid][lane] = static_cast<float>(x);
     __syncwarp();
     float r2 = 0.0f;
     for (int e = lane; e < kD; e += 32) {
