@@ -123,9 +123,9 @@ struct PrefillPlan {
   size_t off_meta, off_cand, bytes;
 };
 
-PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H, int topk) {
+PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H, int topk, int G = 0) {
   PrefillPlan P{};
-  P.G = 256 / H;
+  P.G = G > 0 ? G : 256 / H;
   P.n_groups = static_cast<int>((T_q + P.G - 1) / P.G);
   const int sms = sm_count();
   P.S = 1;
@@ -300,7 +300,7 @@ PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int to
   PrunedPlan P{};
   P.seed = plan_prefill(T_q, n_seed, n_seed - 1, H, topk);
   P.dense = plan_prefill(T_q, T_k, q_offset, H, topk);
-  P.screen = plan_prefill(T_q, T_k, q_offset, kPlanRows, topk);
+  P.screen = plan_prefill(T_q, T_k, q_offset, kPlanRows, topk, kScreenQueries);
   P.refine = plan_decode(static_cast<int>(T_q), topk);
   P.cap_row = pruned_cap_row(T_k, topk);
   P.rec_stride = (topk + 1) & ~1;

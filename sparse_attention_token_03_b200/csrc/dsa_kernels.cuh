@@ -113,6 +113,7 @@ enum ScoreEpilogue : int {
 constexpr int kPlanRows = 16;
 constexpr int kRetained = kPlanRows - 2;
 constexpr int kPlanScalars = 32;
+constexpr int kScreenQueries = 8;  // queries per screening MMA (N = 8 x 16 plan rows)
 
 struct ScoreParams {
   int mode;

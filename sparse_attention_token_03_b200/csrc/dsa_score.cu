@@ -469,25 +469,35 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     // d_neg; C carries the residual, bf16-rounding and fp32 slack terms).  A
     // visible non-seed key survives unless U < tau ("DoSA", step 2: prune only
     // when the bound is strictly below the threshold, keep when unsure).
+    // Each retained head's term is evaluated as (w_i/2) d_i + (w_i/2 + alpha_i/2)
+    // |d_i| (equal in exact arithmetic; two FMAs, the second with an
+    // absolute-value operand); the fp32 rounding of the coefficients and of
+    // the sum lies far inside the 2^-10 S ||k|| part of C.  The coefficients
+    // of this thread's queries stay in registers for the whole unit.
     if constexpr (EG >= 2) regs_inc<regs_epi(EG)>();
     const int e = (warp - score_epi_warp0(EG)) >> 2;
-    const int bar = 1 + e;
-    const int etid = (threadIdx.x - 32 * score_epi_warp0(EG)) & (kEpiThreads - 1);
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
     const int q_lo = e * GQ;
-    float* s_pl = s_w;  // [G][kPlanScalars]
     uint32_t at = 0;
     bool ok = true;
     for (int u = u_begin; ok && u < u_end; u += u_step) {
       const Unit U = unit_geometry<G>(p, u, H);
-      epi_sync(bar);
-      for (int i = etid; i < GQ * kPlanScalars; i += kEpiThreads) {
-        const int qq = q_lo + i / kPlanScalars;
-        s_pl[q_lo * kPlanScalars + i] =
-            (qq < U.rows) ? p.plan_s[(U.row0 + qq) * kPlanScalars + (i % kPlanScalars)] : 0.0f;
+      float c1[GQ][kRetained], c2[GQ][kRetained], cc[GQ], tau[GQ];
+#pragma unroll
+      for (int i = 0; i < GQ; ++i) {
+        const int qq = q_lo + i;
+        const bool on = qq < U.rows;
+        const float* ps = p.plan_s + (U.row0 + (on ? qq : 0)) * kPlanScalars;
+#pragma unroll
+        for (int r = 0; r < kRetained; ++r) {
+          const float w = on ? __ldg(ps + r) : 0.0f, ah = on ? __ldg(ps + kRetained + r) : 0.0f;
+          c1[i][r] = 0.5f * w;
+          c2[i][r] = 0.5f * w + ah;
+        }
+        cc[i] = on ? __ldg(ps + 28) : 0.0f;
+        tau[i] = on ? __ldg(ps + 29) : 0.0f;
       }
-      epi_sync(bar);
       int surv[GQ];
 #pragma unroll
       for (int i = 0; i < GQ; ++i) surv[i] = 0;
@@ -507,21 +517,20 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           if (i + 1 < GQ) tmem_ld16(trow + (i + 1) * H, xb[(i + 1) & 1]);
-          const float* pl = s_pl + (q_lo + i) * kPlanScalars;
           const uint32_t* d = xb[i & 1];
           float ub = 0.0f;
 #pragma unroll
           for (int r = 0; r < kRetained; ++r) {
             const float x = __uint_as_float(d[r]);
-            ub = fmaf(pl[r], fmaxf(x, 0.0f), ub);
-            ub = fmaf(pl[kRetained + r], fabsf(x), ub);
+            ub = fmaf(c1[i][r], x, ub);
+            ub = fmaf(c2[i][r], fabsf(x), ub);
           }
           ub = fmaf(0.5f, __uint_as_float(d[kRetained]), ub);
           ub -= fmaxf(__uint_as_float(d[kRetained + 1]), 0.0f);
-          ub = fmaf(pl[28], kn, ub);
+          ub = fmaf(cc[i], kn, ub);
           const int qq = q_lo + i;
           const bool vis = qq < U.rows && key_local < U.vis_base + qq && !is_seed;
-          const bool keep = vis && !(ub < pl[29]);
+          const bool keep = vis && !(ub < tau[i]);
           const uint32_t word = __ballot_sync(0xFFFFFFFFu, keep);
           if (lane == 0 && qq < U.rows && (key_local >> 5) < p.mask_words)
             p.bitmask[(U.row0 + qq) * p.mask_words + (key_local >> 5)] = word;
@@ -877,10 +886,12 @@ cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tq, const CUte
   return cudaErrorInvalidValue;
 }
 
-// Screening: 16 plan rows per query, 16 queries per MMA (N = 256).
+// Screening: 16 plan rows per query, kScreenQueries = 8 queries per MMA
+// (N = 128), four per epilogue thread so that their bound coefficients fit in
+// registers.
 cudaError_t launch_screen(const CUtensorMap& tplan, const CUtensorMap& tk, const ScoreParams& p,
                           int grid, cudaStream_t stream) {
-  return launch_score_t<kPlanRows, 16, 4, 2, kEpiScreen>(tplan, tk, p, grid, stream);
+  return launch_score_t<kPlanRows, kScreenQueries, 5, 2, kEpiScreen>(tplan, tk, p, grid, stream);
 }
 
 }  // namespace dsa
