@@ -24,6 +24,12 @@
  * Readings where the pages are silent: ties in Top-k are broken by the
  * smaller key index; rows with fewer than k visible keys are padded with
  * index -1 and score -inf; the weights are used as given (no extra scale).
+ *
+ * Pins: every function here is checked by tests/test_oracle_pins.py against
+ * something other than itself (the worked numbers "DeepSeek DSA FLOPs"
+ * prints, a hand-worked example, reductions to a textbook matmul + sort,
+ * linearity and homogeneity, exhaustive selection on tiny inputs, and DoSA
+ * cases where the bound is exact or must hold); none is unpinned.
  */
 #include <math.h>
 #include <stdint.h>
