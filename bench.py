@@ -407,7 +407,9 @@ def main():
     e2e = None
     if not args.no_e2e:
         hq = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-        hk = torch.from_numpy(np.ascontiguousarray(x["k"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        # (decode keeps its key cache on the device; the other paths take keys from the host)
+        hk = (None if wl.kind == "decode" else
+              torch.from_numpy(np.ascontiguousarray(x["k"]).view(np.int16)).view(torch.bfloat16).pin_memory())
         hw = torch.from_numpy(x["w"]).pin_memory()
         hoi = torch.empty(out_idx.shape, dtype=torch.int32).pin_memory()
         hos = torch.empty(out_score.shape, dtype=torch.float32).pin_memory()
@@ -415,7 +417,7 @@ def main():
         if wl.kind == "decode":
             extra["sl"] = torch.from_numpy(x["seq_len"]).pin_memory()
             dsl = torch.empty_like(seq_len)
-        h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4 + (rows * 4 if wl.kind == "decode" else 0)
+        h2d = hq.numel() * 2 + (hk.numel() * 2 if hk is not None else 0) + hw.numel() * 4
         d2h = hoi.numel() * 4 + hos.numel() * 4
         n_e2e = max(3, min(args.steps, 20))
         e_ms = []
@@ -429,6 +431,29 @@ def main():
             def e2e_step():
                 dsa.dsa_index_prefill_host(hq, hw, hk, q_off, wl.topk, out_idx=hoi, out_score=hos,
                                            workspace=hws, device=dev)
+        elif wl.kind == "decode":
+            # a decode step's inputs are the new token's query, head weights and
+            # key per sequence (plus the lengths); the key cache of the earlier
+            # tokens stays resident in HBM, and the new keys are appended to it
+            sl_np = x["seq_len"].astype(np.int64)
+            hnew = torch.from_numpy(np.ascontiguousarray(
+                x["k"][np.arange(rows), np.maximum(sl_np - 1, 0)]).view(np.int16)).view(torch.bfloat16).pin_memory()
+            dq, dw, dnew = torch.empty_like(q), torch.empty_like(w), torch.empty(hnew.shape, dtype=k.dtype, device=dev)
+            kc = k.clone()  # the resident cache the new keys are written into
+            bidx = torch.arange(rows, device=dev)
+            h2d = hq.numel() * 2 + hw.numel() * 4 + rows * 4 + hnew.numel() * 2
+            e2e_api = ("dsa_index_decode with a device-resident key cache: query, weights, lengths "
+                       "and one new key per sequence in, results out (one stream)")
+
+            def e2e_step():
+                dq.copy_(hq, non_blocking=True)
+                dw.copy_(hw, non_blocking=True)
+                dsl.copy_(extra["sl"], non_blocking=True)
+                dnew.copy_(hnew, non_blocking=True)
+                kc[bidx, (dsl.long() - 1).clamp_(min=0)] = dnew  # append this step's keys
+                step(dq, dw, kc, out_idx, out_score, dsl)
+                hoi.copy_(out_idx, non_blocking=True)
+                hos.copy_(out_score, non_blocking=True)
         else:
             dq, dk, dw = torch.empty_like(q), torch.empty_like(k), torch.empty_like(w)
             e2e_api = "copies in, device entry point, copies out (one stream)"
@@ -437,11 +462,7 @@ def main():
                 dq.copy_(hq, non_blocking=True)
                 dk.copy_(hk, non_blocking=True)
                 dw.copy_(hw, non_blocking=True)
-                if wl.kind == "decode":
-                    dsl.copy_(extra["sl"], non_blocking=True)
-                    step(dq, dw, dk, out_idx, out_score, dsl)
-                else:
-                    step(dq, dw, dk, out_idx, out_score)
+                step(dq, dw, dk, out_idx, out_score)
                 hoi.copy_(out_idx, non_blocking=True)
                 hos.copy_(out_score, non_blocking=True)
         for i in range(n_e2e + 2):
