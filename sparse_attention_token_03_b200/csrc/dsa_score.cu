@@ -7,23 +7,31 @@
 // score matrix never reaches HBM (the fused score + Top-k idea that the DoSA
 // write-up, section 04, credits to LiteTopK).
 //
-// Layout of one CTA (192 threads, one CTA per SM, persistent over units):
+// Layout of one CTA (one per SM, persistent over work units):
 //   warp 0  TMA producer: the unit's query tile once (B operand, N = G*H rows
 //           of 128 bf16), then key tiles of 128 keys (A operand) through an
-//           NS-stage ring.
+//           NS-stage ring (refine units gather survivor keys with cp.async).
 //   warp 1  TMEM owner and MMA issuer: per key tile, 8 tcgen05.mma (K = 16
 //           each) into one of two TMEM accumulators of N fp32 columns; keys
 //           sit on the 128 TMEM lanes, (query, head) on the columns.
-//   warps 2-5  epilogue: each thread owns one key (TMEM lane), reads its H
-//           dot products per query with tcgen05.ld, forms the weighted ReLU
-//           head sum in registers (heads in ascending order, fp32 FMA chain
-//           from +0), and appends (score, key) records that pass the row's
-//           running threshold.  When a row's buffer fills up, the epilogue
-//           radix-selects a new threshold and compacts the buffer.
+//   epilogue  EG warpgroups (after warps 0-1 when EG = 1, after a whole
+//           control warpgroup when EG = 2 or 4, with setmaxnreg moving
+//           registers to the epilogue); they split the tile's queries.  Each
+//           thread owns one key (TMEM lane), reads its dot products in
+//           16-column chunks with tcgen05.ld, forms the weighted ReLU head sum
+//           on the FMA pipe (head_acc16: eight fp32 chains in a fixed order)
+//           and appends (score, key) records that pass the row's running
+//           threshold to its warp's region of the candidate buffer.
+//   Every kCheckTiles tiles a warpgroup raises each row's threshold from the
+//   row's score histogram in shared memory and compacts a buffer that could
+//   overflow (one copy pass, or an exact radix select when too many records
+//   share the threshold's bin).  The screen variant (EPI = kEpiScreen)
+//   evaluates the DoSA bound instead and writes a survivor bitmask.
 //
-// The admission rule keeps the selection exact: after a compaction at least
-// k records lie at or above the threshold record, so any later key below it
-// (records order by score, then smaller key first) can never enter the Top-k.
+// The admission rule keeps the selection exact: a threshold is only raised
+// to a value with at least k buffered records at or above it, so any later
+// key below it (records order by score, then smaller key first) can never
+// enter the Top-k.
 #include "dsa_kernels.cuh"
 #include "dsa_ptx.cuh"
 
@@ -32,7 +40,7 @@ namespace dsa {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Block-level helpers for the 128 epilogue threads (named barrier 1).
+// Helpers for the 128 threads of one epilogue warpgroup (named barrier 1 + e).
 // ---------------------------------------------------------------------------
 // Each epilogue warpgroup e synchronises on named barrier 1 + e.
 __device__ __forceinline__ void epi_sync(int bar) { named_bar_sync(bar, kEpiThreads); }
