@@ -176,6 +176,20 @@ def test_decode_ragged_lengths():
                    score_of, f"decode k{topk}")
 
 
+def test_decode_h32_ragged_lengths():
+    # the H = 32 decode kernel (the 128K chunk recipe's heads), ragged caches
+    lens = [2500, 0, 1, 1300, 2047, 700]
+    x = make_decode("chunk_128k_h32", B=len(lens), t_cap=2500, seq_len=lens, seed=13)
+    assert x["H"] == 32
+    for topk in (2048, 100):
+        idx, sc = dsa.dsa_index_decode(bf16(x["q"]), f32(x["w"]), bf16(x["k"]),
+                                       torch.from_numpy(x["seq_len"]).cuda(), topk)
+        torch.cuda.synchronize()
+        oi, osc, amax, score_of = oracle_decode_rows(x, topk)
+        check_rows(idx.cpu().numpy(), sc.cpu().numpy(), oi, osc, amax, x["seq_len"], topk,
+                   score_of, f"decode H32 k{topk}")
+
+
 def test_decode_long_caches_split_across_ctas():
     # few sequences with long caches: each sequence's tiles spread over many
     # CTAs, whose partial candidate lists the final selection merges
