@@ -56,3 +56,30 @@ def test_host_validation_without_gpu():
     # workspace queries reject unsupported shapes with 0
     assert L.dsa_index_prefill_workspace_bytes(4, 4, 48, 128, 8) == 0
     assert L.dsa_index_decode_workspace_bytes(0, 16, 64, 128, 8) == 0
+
+
+def test_host_buffer_prefill_validation_without_gpu():
+    L = dsa.lib()
+    P = ctypes.c_void_p
+    dummy = P(256)
+    # unsupported heads, inconsistent sizes and null pointers fail before any CUDA call
+    assert L.dsa_index_prefill_host(dummy, dummy, dummy, 0, 4, 4, 48, 128, 8, dummy, dummy, dummy, 1 << 30, None) == -2
+    assert L.dsa_index_prefill_host(dummy, dummy, dummy, 3, 4, 4, 64, 128, 8, dummy, dummy, dummy, 1 << 30, None) == -1
+    assert L.dsa_index_prefill_host(None, dummy, dummy, 0, 4, 4, 64, 128, 8, dummy, dummy, dummy, 1 << 30, None) == -1
+    # a workspace below the size query is refused
+    need = L.dsa_index_prefill_host_workspace_bytes(4, 4, 64, 128, 8)
+    assert need > 0
+    assert L.dsa_index_prefill_host(dummy, dummy, dummy, 0, 4, 4, 64, 128, 8, dummy, dummy, dummy, need - 1, None) == -3
+    assert b"workspace" in L.dsa_last_error_string()
+    # an empty chunk is a no-op; unsupported shapes size to 0
+    assert L.dsa_index_prefill_host(None, None, dummy, 0, 0, 4, 64, 128, 8, None, None, None, 0, None) == 0
+    assert L.dsa_index_prefill_host_workspace_bytes(4, 4, 64, 128, 4096) == 0
+
+
+def test_host_buffer_binding_checks_dtypes_without_gpu():
+    import torch
+    q = torch.zeros((4, 64, 128), dtype=torch.float32)
+    w = torch.zeros((4, 64), dtype=torch.float32)
+    k = torch.zeros((4, 128), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        dsa.dsa_index_prefill_host(q, w, k, 0, 8, device="cpu")
