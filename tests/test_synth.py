@@ -55,3 +55,30 @@ def test_decode_shapes_and_lengths():
 def test_random_distinct_keys():
     s = random_distinct_keys(1, 0, 100, 60, exclude=np.arange(10))
     assert len(set(s.tolist())) == 60 and s.min() >= 10 and s.max() < 100
+
+
+def test_recipes_match_their_stated_distributions():
+    # w ~ N(0, 1/8) (variance 1/8); the 1M-chunk recipe draws |N(0, 1/8)| with a
+    # negative sign at probability 0.4
+    x = make_prefill("causal_16k_h64", T_q=2048, T_k=2048, q_offset=0, seed=5)
+    assert abs(float(x["w"].astype(np.float64).var()) - 1.0 / 8.0) < 0.01
+    assert abs(float(x["w"].mean())) < 0.01
+    y = make_prefill("chunk_1m_h64", T_q=2048, T_k=4096, q_offset=2048, seed=6)
+    neg = float((y["w"] < 0).mean())
+    assert abs(neg - 0.4) < 0.02
+    assert abs(float((y["w"].astype(np.float64) ** 2).mean()) - 1.0 / 8.0) < 0.01
+
+
+def test_lowrank_keys_live_near_a_rank_16_subspace():
+    # k = U z + 0.3 e with U (128 x 16): the energy outside the top 16
+    # directions is the isotropic noise, about 0.09 * 112 / (128 + 0.09 * 128)
+    from synth import bf16_bits_to_f32
+    x = make_prefill("causal_16k_h64", T_q=1, T_k=4096, q_offset=4095, seed=8)
+    k = bf16_bits_to_f32(x["k"]).astype(np.float64)
+    s = np.linalg.svd(k, compute_uv=False) ** 2
+    outside = float(s[16:].sum() / s.sum())
+    assert 0.04 < outside < 0.11
+    # the gauss recipe has no such structure
+    g = make_prefill("causal_1k_h64", T_q=1, T_k=1024, q_offset=1023, seed=9)
+    sg = np.linalg.svd(bf16_bits_to_f32(g["k"]).astype(np.float64), compute_uv=False) ** 2
+    assert float(sg[16:].sum() / sg.sum()) > 0.7
