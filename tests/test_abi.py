@@ -83,3 +83,14 @@ def test_host_buffer_binding_checks_dtypes_without_gpu():
     k = torch.zeros((4, 128), dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         dsa.dsa_index_prefill_host(q, w, k, 0, 8, device="cpu")
+
+
+def test_binding_has_the_header_names():
+    # the Python layer is a thin binding with the C ABI's names; the error
+    # string is surfaced through DSAError instead of its own function
+    hdr = (ROOT / "include" / "dsa_index.h").read_text()
+    names = set(re.findall(r"^DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", hdr, flags=re.M))
+    assert "dsa_index_prefill_host" in names and len(names) >= 12
+    missing = sorted(n for n in names - {"dsa_last_error_string"} if not callable(getattr(dsa, n, None)))
+    assert not missing, missing
+    assert set(dsa.__all__) >= names - {"dsa_last_error_string"}
