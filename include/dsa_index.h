@@ -24,11 +24,16 @@
  *    out_score[row][0..topk) fp32 scores, sorted by score descending, ties by
  *    smaller key index; entries past m are idx = -1, score = -inf.
  *  - Scores are fp32: dot products accumulate in fp32 on the tensor cores
- *    from the exact bf16 inputs; the head sum is the fp32 chain
- *    acc = fmaf(w_j, max(dot_j, 0), acc) for j = 0..H-1 from acc = +0.
+ *    from the exact bf16 inputs.  The head sum runs as eight fp32 chains,
+ *    chain c = j mod 8 holding a_c = fmaf(w_j, max(dot_j, 0), a_c) over its
+ *    heads in ascending j from a_c = +0, combined as
+ *    ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7)).  Every entry point
+ *    (dense, decode, pruned) uses this one order, so their scores agree bit
+ *    for bit.
  *  - Supported: d == 128, H in {32, 64}, 1 <= topk <= 2048, key counts
- *    below 2^31.  Inputs must be finite (non-finite inputs never fault or
- *    hang, but their order is unspecified).
+ *    below 2^31.  Inputs must be finite: a pair that scores NaN is never
+ *    selected, and a row with any non-finite pair (NaN or +-inf) has
+ *    unspecified contents; non-finite inputs never fault or hang.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) unless stated otherwise, and returns a status:
  */
@@ -62,7 +67,8 @@ typedef struct dsa_stats {
   int64_t survivor_pairs; /* screened pairs whose bound reached the threshold */
   int64_t refined_pairs;  /* survivor pairs scored exactly with all heads */
   int64_t records;        /* records written for the final selection (seed + refined) */
-  int64_t recovered_rows; /* rows recomputed by the dense path after a capacity overflow */
+  int64_t recovered_rows; /* screened rows recomputed by the dense path (survivor overflow, bad seeds) */
+  int64_t bypassed_rows;  /* rows the probe sent to the dense path without screening */
 } dsa_stats;
 
 /* Text of the last error seen by this library in the calling thread. */
@@ -142,18 +148,28 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
  *      U < tau are pruned (strictly; a key whose bound is uncertain is kept).
  *   3. Survivors are scored exactly with all heads; records at or above the
  *      row's topk-th seed record enter the final exact Top-k with the seeds'.
+ * The first 64 rows of a chunk longer than 128 rows are a probe: they
+ * always take steps 1-3, and from their survivor counts the device estimates
+ * whether pruning pays for this chunk (screen, seed and refine costs against
+ * a dense pass).  If it does not, the remaining rows skip steps 1-3 and go
+ * straight to the dense kernel, so the call costs little more than
+ * dsa_index_prefill on inputs the bound cannot filter.  Rows whose survivors
+ * exceed a list of max(T_k / 16, 4 topk) keys are also recomputed densely.
+ * The decision is taken on the device: the call never waits for the host.
  *   seed_idx   device, [n_seed] int32: distinct keys with 0 <= seed < q_offset
  *              (visible to every row); topk <= n_seed <= q_offset, else
  *              DSA_ESEED before any launch.  Out-of-range or repeated seeds
  *              found on the device make every row fall back to the exact
  *              dense computation (reported as DSA_ESEED when stats is given).
  *   stats      host, may be NULL: when given, the call synchronises `stream`
- *              and fills the counters (screened_pairs: visible non-seed
- *              pairs; survivor_pairs: pairs with U >= tau; refined_pairs:
- *              survivors scored exactly; records: seed Top-k + refined
- *              records; recovered_rows: rows recomputed densely because
- *              their survivors exceeded the per-row list capacity of
- *              max(T_k / 4, 4 topk) keys).
+ *              and fills the counters, over the rows that were screened
+ *              (screened_pairs: their visible non-seed pairs; survivor_pairs:
+ *              pairs with U >= tau; refined_pairs: survivors scored exactly;
+ *              records: seed Top-k + refined candidates read by the final
+ *              selection of the rows it finished; recovered_rows: screened
+ *              rows recomputed densely after a survivor overflow or a bad
+ *              seed list) and bypassed_rows (rows sent to the dense kernel
+ *              without screening).
  * Requires T_q <= 65536.  The workspace is sized by
  * dsa_index_prefill_pruned_workspace_bytes().
  */
@@ -166,6 +182,25 @@ DSA_API int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const ui
                                      size_t ws_bytes, void* stream);
 
 /*
+ * Diagnostics of the most recent dsa_index_prefill_pruned call that used
+ * `workspace` with the same sizes ("DoSA", step 2: the screen's survivor
+ * decisions).  Copies, on `stream`:
+ *   mask       device, [T_q][ceil(T_k / 32)] uint32: bit s % 32 of word s / 32
+ *              of row t is 1 when the screen kept key s (U >= tau), 0 when it
+ *              pruned it.  Defined for screened rows, keys 0..q_offset+t;
+ *              seed keys read 0 (they are scored exactly, never screened).
+ *   tau        device, [T_q] fp32: the row's topk-th seed score.
+ *   row_state  device, [T_q] int32: 0 screened and refined, 1 screened and
+ *              recomputed densely (survivor overflow), 2 not screened
+ *              (the probe's bypass), 3 bad seed list.
+ * For tests of the bound's safety: a pruned key must score below tau.
+ */
+DSA_API int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_q, int64_t T_k,
+                                               int64_t q_offset, int H, int d, int topk, int n_seed,
+                                               uint32_t* mask, float* tau, int32_t* row_state,
+                                               void* stream);
+
+/*
  * Batched decode that allocates nothing (no counterpart in the paper; a
  * library convenience).  Same computation, arguments and outputs as
  * dsa_index_decode, without the workspace: for callers that cannot hand the
@@ -174,22 +209,37 @@ DSA_API int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const ui
  * not call cudaMalloc on a latency-critical path because it can synchronise
  * the device.
  *  - Scratch is a fixed array in the library's device image, sized for at
- *    most 64 sequences at topk <= 2048 (about 28 MB).  Every GPU on which the
- *    library is loaded holds that memory until the process exits.  B > 64
- *    returns DSA_EINVAL with an explanatory message; nothing is launched.
+ *    most 64 sequences at topk <= 2048 (36,827,136 bytes, about 37 MB).
+ *    Every GPU on which the library is loaded holds that memory until the
+ *    process exits.  B > 64 returns DSA_EINVAL with an explanatory message;
+ *    nothing is launched.
  *  - The call itself allocates no device memory: no cudaMalloc/cudaFree, no
- *    allocating library routine.  The first call on each device looks up the
- *    scratch's device address (with that device current); make that first
- *    call before any stream capture.
+ *    allocating library routine.  Each call looks up the scratch's device
+ *    address on the current device (cudaGetSymbolAddress; the first lookup
+ *    on a device loads the library's kernels there), so make the first call
+ *    on each device before any stream capture.
  *  - All calls share the one scratch array, which keeps the last call's
  *    contents; each call initialises what it reads.  Calls whose executions
  *    overlap on the GPU (different streams, or host threads racing on the
  *    same device) race on the scratch and give undefined results: serialise
  *    them.
+ *  - Device-side checks (a length outside [0, t_cap], a bounded wait that
+ *    gave up, a non-finite pair) set the status word at the start of the
+ *    static scratch, not in a caller workspace: read it with
+ *    dsa_index_decode_noalloc_status().
  */
 DSA_API int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const uint16_t* k_cache,
                                      const int32_t* seq_len, int B, int64_t t_cap, int H, int d,
                                      int topk, int32_t* out_idx, float* out_score, void* stream);
+
+/*
+ * Device status word of the most recent dsa_index_decode_noalloc call on the
+ * current device (the word at the start of the library's static scratch;
+ * bits as for dsa_index_device_status below).  Synchronises `stream`; it
+ * allocates nothing.  No counterpart in the paper: the status reader of the
+ * allocation-free decode.
+ */
+DSA_API int dsa_index_decode_noalloc_status(uint32_t* status, void* stream);
 
 /*
  * Device status word of the most recent call that used `workspace`: 0 when
@@ -197,10 +247,22 @@ DSA_API int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const ui
  * Bit 0: a bounded wait inside a kernel gave up (the kernel unwound).
  * Bit 1: a capacity or length check failed.  Bit 2: the seed list was invalid.
  * Bit 3: a causally visible (query, key) pair scored inf or NaN, i.e. q, k or
- * w holds a non-finite value; such pairs are never selected and the rows
- * they belong to are unspecified.
+ * w holds a non-finite value; NaN pairs are never selected and the rows with
+ * a non-finite pair are unspecified.
  */
 DSA_API int dsa_index_device_status(const void* workspace, uint32_t* status, void* stream);
+
+/*
+ * Failure injection for tests of the bounded device waits (no counterpart on
+ * the pages).  Arms a one-shot fault for the calling host thread: the next
+ * fused scoring launch of any entry point issues no loads, so its MMA warp
+ * waits for data that never arrives; that wait gives up after limit_ns
+ * (1 ms .. 2 s), the kernel unwinds (in-flight copies and tensor-core work
+ * drained, tensor memory released), sets bit 0 of the device status word and
+ * returns.  The call's outputs are then unspecified; later calls are
+ * unaffected.  Nothing faults or hangs: every wait in the library is bounded.
+ */
+DSA_API int dsa_test_inject_wait_timeout(int64_t limit_ns);
 
 /*
  * Per-kernel timing of the calling thread's entry-point calls (for

@@ -42,7 +42,6 @@ def _load():
         D = ctypes.c_double
         _lib.oracle_row_scores.argtypes = [P, P, P, I64, I32, I32, P]
         _lib.oracle_score_pairs.argtypes = [P, P, P, I32, I32, I64, P, P, P, I32]
-        _lib.oracle_topk_of_scores.argtypes = [P, I64, I32, P, P]
         _lib.oracle_prefill_topk.argtypes = [P, P, P, I64, I64, I64, I32, I32, I32, P, I64,
                                              P, P, P, P, I32]
         _lib.oracle_prefill_topk.restype = I32
@@ -100,14 +99,6 @@ def score_pairs(q, w, k, q_rows, keys, n_threads: int | None = None) -> np.ndarr
     _load().oracle_score_pairs(_p(q), _p(w), _p(k), H, d, q_rows.shape[0], _p(q_rows),
                                _p(keys), _p(out), n_threads or threads())
     return out
-
-
-def topk_of_scores(scores, topk: int):
-    scores = _c(scores, np.float64)
-    idx = np.empty(topk, np.int32)
-    sc = np.empty(topk, np.float64)
-    _load().oracle_topk_of_scores(_p(scores), scores.shape[0], topk, _p(idx), _p(sc))
-    return idx, sc
 
 
 def prefill_topk(q, w, k, q_offset: int, topk: int, rows=None, want_scores: bool = False,

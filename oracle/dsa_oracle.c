@@ -26,10 +26,14 @@
  * index -1 and score -inf; the weights are used as given (no extra scale).
  *
  * Pins: every function here is checked by tests/test_oracle_pins.py against
- * something other than itself (the worked numbers "DeepSeek DSA FLOPs"
- * prints, a hand-worked example, reductions to a textbook matmul + sort,
- * linearity and homogeneity, exhaustive selection on tiny inputs, and DoSA
- * cases where the bound is exact or must hold); none is unpinned.
+ * something other than itself: the worked numbers "DeepSeek DSA FLOPs"
+ * prints, a hand-worked example, reductions to a textbook matmul + sort
+ * (numpy), linearity and homogeneity, exhaustive selection on tiny inputs,
+ * the planner sample positions the DoSA notes print, and DoSA cases where the
+ * bound is exact or must hold.  oracle_score_pairs is pinned against a numpy
+ * matmul of the widened inputs at random (row, key) pairs of chunked and
+ * decode layouts.  Parity is unpinned only for the per-element fp32 results
+ * of the GPU beyond the stated tolerance.
  */
 #include <math.h>
 #include <stdint.h>
@@ -120,17 +124,6 @@ static void emit_topk(rec_t *recs, int64_t n, int topk, int32_t *out_idx,
       out_score[i] = -INFINITY;
     }
   }
-}
-
-OR_API void oracle_topk_of_scores(const double *scores, int64_t n, int topk,
-                                  int32_t *out_idx, double *out_score) {
-  rec_t *recs = (rec_t *)malloc(sizeof(rec_t) * (size_t)(n > 0 ? n : 1));
-  for (int64_t s = 0; s < n; ++s) {
-    recs[s].score = scores[s];
-    recs[s].key = s;
-  }
-  emit_topk(recs, n, topk, out_idx, out_score);
-  free(recs);
 }
 
 /* ---------------------------------------------------------------------------
@@ -380,11 +373,16 @@ OR_API double oracle_dosa_bound(const double *plan, const uint16_t *q_row,
   return U;
 }
 
-/* Evenly spaced planner sample of the seed list: entry (2i+1)*n/(2m) for
- * i < m = min(128, n). */
+/* Planner sample of the seed list ("DoSA" reading notes, annotation
+ * ADQKPC5Q, step 1: 128 positions 32 + 64 i of the seed region).  Reading:
+ * the midpoints of 128 equal slices of the first n' = min(n_seed, 8192) seed
+ * entries, entry floor((2i+1) n' / (2m)) for i < m = min(128, n'); at
+ * n' = 8192 these are exactly the positions 32 + 64 i, and shorter seed
+ * lists keep the same even spacing. */
 OR_API int oracle_dosa_sample(const int32_t *seeds, int n_seed, int32_t *out) {
-  int m = n_seed < 128 ? n_seed : 128;
-  for (int i = 0; i < m; ++i) out[i] = seeds[((int64_t)(2 * i + 1) * n_seed) / (2 * m)];
+  int n = n_seed < 8192 ? n_seed : 8192;
+  int m = n < 128 ? n : 128;
+  for (int i = 0; i < m; ++i) out[i] = seeds[((int64_t)(2 * i + 1) * n) / (2 * m)];
   return m;
 }
 

@@ -20,8 +20,9 @@ __all__ = [
     "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
-    "dsa_index_decode_noalloc", "dsa_index_prefill_pruned", "dsa_index_prefill_pruned_workspace_bytes",
-    "dsa_index_prefill_host", "dsa_index_prefill_host_workspace_bytes",
+    "dsa_index_decode_noalloc", "dsa_index_decode_noalloc_status", "dsa_index_prefill_pruned",
+    "dsa_index_prefill_pruned_workspace_bytes", "dsa_index_prefill_pruned_survivors",
+    "dsa_index_prefill_host", "dsa_index_prefill_host_workspace_bytes", "dsa_test_inject_wait_timeout",
 ]
 
 DSA_OK = 0
@@ -68,10 +69,16 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_prefill_pruned_workspace_bytes.restype = SZ
         L.dsa_index_prefill_pruned.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I, P, P, P, P, SZ, P]
         L.dsa_index_prefill_pruned.restype = I
+        L.dsa_index_prefill_pruned_survivors.argtypes = [P, I64, I64, I64, I, I, I, I, P, P, P, P]
+        L.dsa_index_prefill_pruned_survivors.restype = I
         L.dsa_index_decode_noalloc.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P]
         L.dsa_index_decode_noalloc.restype = I
+        L.dsa_index_decode_noalloc_status.argtypes = [P, P]
+        L.dsa_index_decode_noalloc_status.restype = I
         L.dsa_index_device_status.argtypes = [P, P, P]
         L.dsa_index_device_status.restype = I
+        L.dsa_test_inject_wait_timeout.argtypes = [I64]
+        L.dsa_test_inject_wait_timeout.restype = I
         L.dsa_profile_enable.argtypes = [I]
         L.dsa_profile_enable.restype = I
         L.dsa_profile_read.argtypes = [P, P, I, P]
@@ -209,7 +216,7 @@ def dsa_index_prefill_host(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_
 class _Stats(ctypes.Structure):
     _fields_ = [("screened_pairs", ctypes.c_int64), ("survivor_pairs", ctypes.c_int64),
                 ("refined_pairs", ctypes.c_int64), ("records", ctypes.c_int64),
-                ("recovered_rows", ctypes.c_int64)]
+                ("recovered_rows", ctypes.c_int64), ("bypassed_rows", ctypes.c_int64)]
 
 
 def dsa_index_prefill_pruned_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int,
@@ -249,6 +256,25 @@ def dsa_index_prefill_pruned(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, 
     if stats:
         return out_idx, out_score, {f: int(getattr(st, f)) for f, _ in _Stats._fields_}
     return out_idx, out_score
+
+
+def dsa_index_prefill_pruned_survivors(workspace: torch.Tensor, T_q: int, T_k: int, q_offset: int, H: int,
+                                       d: int, topk: int, n_seed: int):
+    """The screen's decisions of the last pruned call on `workspace` (same sizes).
+
+    Returns (mask (T_q, ceil(T_k/32)) int32 bit words, tau (T_q,) fp32,
+    row_state (T_q,) int32) on the workspace's device.
+    """
+    dev = workspace.device
+    _need(workspace, "workspace", torch.uint8, 1, dev)
+    mask = torch.empty((T_q, (T_k + 31) // 32), dtype=torch.int32, device=dev)
+    tau = torch.empty(T_q, dtype=torch.float32, device=dev)
+    state = torch.empty(T_q, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_pruned_survivors(workspace.data_ptr(), T_q, T_k, int(q_offset), H, d,
+                                                        int(topk), int(n_seed), mask.data_ptr(),
+                                                        tau.data_ptr(), state.data_ptr(), _stream_ptr(dev)))
+    return mask, tau, state
 
 
 def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
@@ -302,6 +328,23 @@ def dsa_index_decode_noalloc(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Te
     return out_idx, out_score
 
 
+def dsa_index_decode_noalloc_status(device=None) -> int:
+    """Device status word of the last dsa_index_decode_noalloc call on
+    ``device`` (default: the current CUDA device); synchronises its current
+    stream and allocates nothing."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_decode_noalloc_status(ctypes.byref(st), _stream_ptr(dev)))
+    return int(st.value)
+
+
+def dsa_test_inject_wait_timeout(limit_ns: int) -> None:
+    """Arm a one-shot injected wait timeout for the calling thread's next
+    scoring launch (tests of the bounded-wait failure path)."""
+    _check(lib().dsa_test_inject_wait_timeout(int(limit_ns)))
+
+
 def dsa_profile_enable(on: bool = True) -> None:
     """Record per-kernel CUDA events inside the library's entry points."""
     _check(lib().dsa_profile_enable(1 if on else 0))
@@ -309,11 +352,11 @@ def dsa_profile_enable(on: bool = True) -> None:
 
 def dsa_profile_read() -> list[tuple[str, float]]:
     """(kernel name, device ms) for each kernel of the calling thread's last call."""
-    ms = (ctypes.c_float * 16)()
-    names = (ctypes.c_char_p * 16)()
+    ms = (ctypes.c_float * 32)()
+    names = (ctypes.c_char_p * 32)()
     n = ctypes.c_int(0)
-    _check(lib().dsa_profile_read(ms, names, 16, ctypes.byref(n)))
-    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, 16))]
+    _check(lib().dsa_profile_read(ms, names, 32, ctypes.byref(n)))
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, 32))]
 
 
 def dsa_index_device_status(workspace: torch.Tensor) -> int:

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -66,23 +67,29 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
 }
 
 int sm_count() {
-  static int cached[64] = {};
+  // per-device cache; host threads may race on it harmlessly (atomic, and
+  // every writer stores the same value)
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 64 && cached[dev]) return cached[dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 148;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  if (dev < 64) cached[dev] = n;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 // Optional per-kernel timing: when enabled, every entry point records a CUDA
 // event on its stream before its first launch and after each launch.
+constexpr int kProfileEvents = 32;
 struct Profile {
   bool enabled = false;
   int n = 0;
-  cudaEvent_t ev[16] = {};
-  const char* name[16] = {};
+  cudaEvent_t ev[kProfileEvents] = {};
+  const char* name[kProfileEvents] = {};
 };
 thread_local Profile g_prof;
 
@@ -96,13 +103,22 @@ void prof_begin(cudaStream_t st) {
 }
 
 void prof_mark(cudaStream_t st, const char* kernel) {
-  if (!g_prof.enabled || g_prof.n >= 16) return;
+  if (!g_prof.enabled || g_prof.n >= kProfileEvents) return;
   cudaEvent_t& e = g_prof.ev[g_prof.n];
   if (!e) cudaEventCreate(&e);
   cudaEventRecord(e, st);
   g_prof.name[g_prof.n] = kernel;
   ++g_prof.n;
 }
+
+// One-shot failure injection armed by dsa_test_inject_wait_timeout (per
+// host thread): the next fused-kernel launch withholds its loads and limits
+// its pipeline waits, so that a wait runs out on the device.
+struct WaitInjection {
+  bool armed = false;
+  uint64_t limit_ns = 0;
+};
+thread_local WaitInjection g_inject;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -123,7 +139,8 @@ struct PrefillPlan {
   size_t off_meta, off_cand, bytes;
 };
 
-PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H, int topk, int G = 0) {
+PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H, int topk, int G = 0,
+                         int max_s = 64) {
   PrefillPlan P{};
   P.G = G > 0 ? G : 256 / H;
   P.n_groups = static_cast<int>((T_q + P.G - 1) / P.G);
@@ -135,7 +152,7 @@ PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H,
     const int64_t tiles = (min_keys + kTileKeys - 1) / kTileKeys;
     const int want = (sms + P.n_groups - 1) / P.n_groups;
     P.S = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, tiles / 16)));
-    P.S = std::min(P.S, 64);
+    P.S = std::min(P.S, std::max(max_s, 1));
   }
   P.n_units = P.n_groups * P.S;
   // Epilogue width: four warpgroups (one query each at H = 64) hide the
@@ -275,32 +292,47 @@ int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const
 
 // ---------------------------------------------------------------------------
 // Workspace of the pruned (DoSA) prefill.
+//
+// The chunk's first probe rows always take the pruned path; from their
+// survivor counts a device-side decision (decide_kernel) either lets the
+// remaining rows take it too or marks them for the dense pass, so that the
+// call never costs much more than the dense one on inputs where the bound
+// filters little.  Nothing synchronises with the host.
 // ---------------------------------------------------------------------------
+constexpr int64_t kProbeRows = 64;  // a multiple of every query group size (4, 8)
+
 struct PrunedPlan {
-  PrefillPlan seed;    // seed scoring: gathered seed keys, all visible
-  PrefillPlan dense;   // exact dense recovery of flagged rows
-  PrefillPlan screen;  // screening geometry (16 plan rows per query)
-  DecodePlan refine;   // refine: one "sequence" of survivors per row
-  int cap_row;         // survivor ids kept per row
-  int rec_stride;      // seed records per row (topk rounded up to even)
+  int64_t probe;          // rows of the probe (all rows of a short chunk)
+  PrefillPlan seed[2];    // seed scoring of the probe rows / the remaining rows
+  PrefillPlan screen[2];  // screening geometry (16 plan rows per query), same split
+  PrefillPlan dense;      // exact dense pass over flagged rows
+  DecodePlan refine;      // refine: one "sequence" of survivors per row
+  int cap_row;            // survivor ids kept per row
+  int rec_stride;         // seed records per row (topk rounded up to even)
   int64_t mask_words;
-  size_t off_stats, off_seed_bits, off_k_seed, off_cand, off_seed_rec, off_tau, off_plan_q, off_plan_s,
+  size_t off_stats, off_ctl, off_seed_bits, off_k_seed, off_cand, off_seed_rec, off_tau, off_plan_q, off_plan_s,
       off_knorm, off_bitmask, off_surv_count, off_surv_ids, off_refine_len, off_row_flags, off_init_thr,
       off_refine, bytes;
 };
 
 int pruned_cap_row(int64_t T_k, int topk) {
-  // survivor lists hold up to a quarter of the keys (rows with more survivors
-  // than that are recomputed by the dense path)
-  const int64_t c = std::max<int64_t>(T_k / 4, 4 * static_cast<int64_t>(topk));
+  // survivor lists hold up to a sixteenth of the keys: a row with more
+  // survivors is cheaper to recompute densely than to refine key by key
+  const int64_t c = std::max<int64_t>(T_k / 16, 4 * static_cast<int64_t>(topk));
   return static_cast<int>(std::min<int64_t>(std::min<int64_t>(c, T_k), int64_t(1) << 30));
 }
 
 PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int topk, int n_seed) {
   PrunedPlan P{};
-  P.seed = plan_prefill(T_q, n_seed, n_seed - 1, H, topk);
+  P.probe = T_q > 2 * kProbeRows ? kProbeRows : T_q;
+  const int64_t rows[2] = {P.probe, T_q - P.probe};
+  for (int i = 0; i < 2; ++i) {
+    // a seed-scoring split needs a few times topk keys, or its streaming
+    // threshold never rises and the seed select merges every seed record
+    P.seed[i] = plan_prefill(rows[i], n_seed, n_seed - 1, H, topk, 0, n_seed / (2 * topk));
+    P.screen[i] = plan_prefill(rows[i], T_k, q_offset + (i ? P.probe : 0), kPlanRows, topk, kScreenQueries);
+  }
   P.dense = plan_prefill(T_q, T_k, q_offset, H, topk);
-  P.screen = plan_prefill(T_q, T_k, q_offset, kPlanRows, topk, kScreenQueries);
   P.refine = plan_decode(static_cast<int>(T_q), topk);
   P.cap_row = pruned_cap_row(T_k, topk);
   P.rec_stride = (topk + 1) & ~1;
@@ -312,11 +344,11 @@ PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int to
     return o;
   };
   P.off_stats = take(8 * sizeof(unsigned long long));
+  P.off_ctl = take(8 * sizeof(uint32_t));
   P.off_seed_bits = take(static_cast<size_t>(P.mask_words) * 4);
   P.off_k_seed = take(static_cast<size_t>(n_seed) * kD * 2);
-  // seed scoring and dense recovery run at different times and share one area
-  const size_t sb = P.seed.bytes, db = P.dense.bytes;
-  P.off_cand = take(std::max(sb, db));
+  // seed scoring and the dense pass run at different times and share one area
+  P.off_cand = take(std::max({P.seed[0].bytes, P.seed[1].bytes, P.dense.bytes}));
   P.off_seed_rec = take(static_cast<size_t>(T_q) * P.rec_stride * 8);
   P.off_tau = take(static_cast<size_t>(T_q) * 4);
   P.off_plan_q = take(static_cast<size_t>(T_q) * kPlanRows * kD * 2);
@@ -333,37 +365,126 @@ PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int to
   return P;
 }
 
+// Seed scoring, plan, screen and compaction of the n rows starting at r0 of
+// a pruned call (i = 0: the probe rows, i = 1: the rest of the chunk).
+// skip (device, may be null): every launch does nothing while the word is set.
+int pruned_rows(const PrunedPlan& P, int i, int64_t r0, int64_t n, const uint16_t* q, const float* w,
+                int64_t q_offset, int64_t T_k, int H, int topk, const int32_t* seed_idx, int n_seed,
+                const CUtensorMap& tk, uint8_t* ws, const uint32_t* skip, cudaStream_t st) {
+  if (n <= 0) return DSA_OK;
+  int rc;
+  cudaError_t e;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  auto at = [&](size_t off) { return ws + off; };
+  const uint16_t* qr = q + static_cast<size_t>(r0) * H * kD;
+  const float* wr = w + static_cast<size_t>(r0) * H;
+  const PrefillPlan& SP = P.seed[i];
+  const PrefillPlan& CP = P.screen[i];
+  float* tau = reinterpret_cast<float*>(at(P.off_tau)) + r0;
+  uint64_t* seed_rec = reinterpret_cast<uint64_t*>(at(P.off_seed_rec)) + r0 * P.rec_stride;
+  uint16_t* plan_q = reinterpret_cast<uint16_t*>(at(P.off_plan_q)) + r0 * kPlanRows * kD;
+  float* plan_s = reinterpret_cast<float*>(at(P.off_plan_s)) + r0 * kPlanScalars;
+  uint32_t* bitmask = reinterpret_cast<uint32_t*>(at(P.off_bitmask)) + r0 * P.mask_words;
+  int32_t* surv_count = reinterpret_cast<int32_t*>(at(P.off_surv_count)) + r0;
+  CUtensorMap tq, tks, tplan;
+  if ((rc = make_tmap(&tq, qr, n * H, SP.G * H)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tks, at(P.off_k_seed), n_seed, kTileKeys)) != DSA_OK) return rc;
+  if ((rc = make_tmap(&tplan, plan_q, n * kPlanRows, CP.G * kPlanRows)) != DSA_OK) return rc;
+  // seed scores with all heads; per row: sorted seed Top-k records and tau
+  ScoreParams s1{};
+  s1.mode = kModeGathered;
+  s1.topk = topk;
+  s1.lay = SP.lay;
+  s1.S = SP.S;
+  s1.n_groups = SP.n_groups;
+  s1.n_units = SP.n_units;
+  s1.T_q = n;
+  s1.T_k = n_seed;
+  s1.w = wr;
+  s1.key_ids = seed_idx;
+  s1.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + SP.off_cand));
+  s1.meta = reinterpret_cast<int32_t*>(at(P.off_cand + SP.off_meta));
+  s1.err = err;
+  s1.skip = skip;
+  if ((e = launch_score(H, SP.G, SP.eg, tq, tks, s1, SP.grid, st)) != cudaSuccess)
+    return cuda_fail(e, "seed score launch");
+  prof_mark(st, "seed_score");
+  SelectParams s2{};
+  s2.mode = kModePrefill;
+  s2.G = SP.G;
+  s2.S = SP.S;
+  s2.topk = topk;
+  s2.lay = SP.lay;
+  s2.n_rows = n;
+  s2.cand = s1.cand;
+  s2.meta = s1.meta;
+  s2.out_rec = seed_rec;
+  s2.rec_stride = P.rec_stride;
+  s2.out_kth = tau;
+  s2.err = err;
+  s2.skip = skip;
+  if ((e = launch_select(s2, st)) != cudaSuccess) return cuda_fail(e, "seed select launch");
+  prof_mark(st, "seed_select");
+  // screening plan per row
+  PlanParams pp{qr, wr, reinterpret_cast<const uint16_t*>(at(P.off_k_seed)), n_seed, n, tau, plan_q, plan_s, skip};
+  if ((e = launch_plan(H, pp, st)) != cudaSuccess) return cuda_fail(e, "plan launch");
+  prof_mark(st, "plan");
+  // screen every visible non-seed key: bound -> survivor bitmask
+  ScoreParams s3{};
+  s3.mode = kModePrefill;
+  s3.topk = topk;
+  s3.lay = CP.lay;
+  s3.S = CP.S;
+  s3.n_groups = CP.n_groups;
+  s3.n_units = CP.n_units;
+  s3.q_offset = q_offset + r0;
+  s3.T_q = n;
+  s3.T_k = T_k;
+  s3.err = err;
+  s3.plan_s = plan_s;
+  s3.knorm = reinterpret_cast<const float*>(at(P.off_knorm));
+  s3.seed_bits = reinterpret_cast<const uint32_t*>(at(P.off_seed_bits));
+  s3.bitmask = bitmask;
+  s3.mask_words = P.mask_words;
+  s3.surv_count = surv_count;
+  s3.skip = skip;
+  if ((e = launch_screen(tplan, tk, s3, CP.grid, st)) != cudaSuccess) return cuda_fail(e, "screen launch");
+  prof_mark(st, "screen");
+  // survivors -> id lists; rows whose survivors overflow are flagged
+  CompactParams cp{n, q_offset + r0, topk, bitmask, P.mask_words, surv_count, P.cap_row,
+                   reinterpret_cast<int32_t*>(at(P.off_surv_ids)) + r0 * P.cap_row,
+                   reinterpret_cast<int32_t*>(at(P.off_refine_len)) + r0,
+                   reinterpret_cast<int32_t*>(at(P.off_row_flags)) + r0, seed_rec, P.rec_stride,
+                   reinterpret_cast<uint64_t*>(at(P.off_init_thr)) + r0, err, skip};
+  if ((e = launch_compact(cp, st)) != cudaSuccess) return cuda_fail(e, "compact launch");
+  prof_mark(st, "compact");
+  return DSA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Scratch for dsa_index_decode_noalloc.  The array lives in the library's
 // device image, so every GPU on which the library's kernels are loaded holds
-// it (about 28 MB) until the process exits.  Host code must not hand the
-// symbol itself to a kernel: on the host it only names a stand-in; the device
-// address comes from cudaGetSymbolAddress, once per device.
+// it (36,827,136 bytes, about 37 MB) until the process exits.  Host code must
+// not hand the symbol itself to a kernel: on the host it only names a
+// stand-in; the device address comes from cudaGetSymbolAddress, looked up on
+// every call with the caller's device current (cheap, not a stream
+// operation), so that a context that was torn down and re-created never
+// leaves a stale address behind.
 // ---------------------------------------------------------------------------
 constexpr int kNoAllocMaxB = 64;      // largest batch served from the static scratch
 constexpr int kNoAllocMaxGrid = 160;  // persistent CTAs used by that path (<= SMs)
 constexpr size_t kNoAllocScratchBytes = plan_decode_layout(kNoAllocMaxB, kMaxTopk, kNoAllocMaxGrid).bytes;
+// the header states this size; keep the two in step
+static_assert(kNoAllocScratchBytes == 36827136, "static decode scratch size changed: update dsa_index.h");
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
-
-// Device address of the static scratch on the current device (looked up on
-// the first call per device, with that device current).
+// Device address of the static scratch on the current device.
 int noalloc_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(DSA_EUNSUPPORTED, "device index %d above 63", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+  *out = p;
   return DSA_OK;
 }
 
@@ -379,17 +500,18 @@ int check_prefill_args(int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d,
 
 // Fused score + streaming Top-k over the chunk's rows, then the final
 // selection, on device buffers (arguments already checked).  reset_status
-// clears the workspace's device status word first.
+// clears the workspace's device status word first; begin_profile starts the
+// per-kernel events, profile records them.
 int prefill_run(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset, int64_t T_q,
                 int64_t T_k, int H, int topk, int32_t* out_idx, float* out_score, uint8_t* ws,
-                const PrefillPlan& P, bool reset_status, bool profile, cudaStream_t st) {
+                const PrefillPlan& P, bool reset_status, bool begin_profile, bool profile, cudaStream_t st) {
   int rc;
   CUtensorMap tq, tk;
   if ((rc = make_tmap(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
   if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
   cudaError_t e;
   if (reset_status && (e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  if (profile) prof_begin(st);
+  if (begin_profile) prof_begin(st);
 
   ScoreParams sp{};
   sp.mode = kModePrefill;
@@ -423,6 +545,31 @@ int prefill_run(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_
   if ((e = launch_select(se, st)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
   if (profile) prof_mark(st, "select_topk");
   return DSA_OK;
+}
+
+// Row blocks of a large prefill.  A chunk whose candidate buffers would not
+// fit the caller's workspace runs as consecutive launches over row blocks
+// (rows are independent, so the result is the same bit for bit); the
+// workspace size query caps its answer at kPrefillWorkspaceCap.
+constexpr size_t kPrefillWorkspaceCap = size_t(4) << 30;
+
+// Workspace of a launch over `rows` rows, sized for the most key splits any
+// offset can give them (q_offset = T_k - rows).
+size_t block_bytes(int64_t rows, int64_t T_k, int H, int topk) {
+  return plan_prefill(rows, T_k, std::max<int64_t>(T_k - rows, 0), H, topk).bytes;
+}
+
+// Largest row count (all rows, or a multiple of the query group) whose launch
+// fits `bytes`; 0 when not even one group fits.
+int64_t prefill_block_rows(int64_t T_q, int64_t T_k, int H, int topk, size_t bytes) {
+  if (block_bytes(T_q, T_k, H, topk) <= bytes) return T_q;
+  const int64_t G = 256 / H;
+  int64_t lo = 0, hi = (T_q - 1) / G;  // in groups
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (block_bytes(mid * G, T_k, H, topk) <= bytes) lo = mid; else hi = mid - 1;
+  }
+  return lo * G;
 }
 
 // ------------------------------------------------------- host-buffer prefill
@@ -497,14 +644,34 @@ int host_streams(HostStreams** out) {
 
 }  // namespace
 
+namespace dsa {
+void take_wait_injection(ScoreParams& p) {
+  if (!g_inject.armed) return;
+  g_inject.armed = false;
+  p.stall_loads = 1;
+  p.wait_ns = g_inject.limit_ns;
+}
+}  // namespace dsa
+
 extern "C" {
+
+int dsa_test_inject_wait_timeout(int64_t limit_ns) {
+  if (limit_ns < 1000000 || limit_ns > 2000000000)
+    return fail(DSA_EINVAL, "limit_ns = %lld outside [1 ms, 2 s]", static_cast<long long>(limit_ns));
+  g_inject.armed = true;
+  g_inject.limit_ns = static_cast<uint64_t>(limit_ns);
+  return DSA_OK;
+}
+
 
 const char* dsa_last_error_string(void) { return g_last_error.c_str(); }
 
 size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
   if (check_shape(H, d, topk) != DSA_OK || T_q < 0 || T_k < 1) return 0;
-  // the split choice depends on q_offset; size for the most splits (q_offset = T_k - T_q)
-  return plan_prefill(T_q, T_k, T_k - T_q, H, topk).bytes;
+  const size_t full = block_bytes(T_q, T_k, H, topk);
+  if (full <= kPrefillWorkspaceCap) return full;
+  // larger chunks run in row blocks whose workspace fits the cap
+  return block_bytes(prefill_block_rows(T_q, T_k, H, topk, kPrefillWorkspaceCap), T_k, H, topk);
 }
 
 int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
@@ -517,12 +684,23 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
       !aligned(out_idx, 4) || !aligned(out_score, 4))
     return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
-  const size_t need = dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk);
-  const PrefillPlan P = plan_prefill(T_q, T_k, q_offset, H, topk);
-  if (ws_bytes < std::max(need, P.bytes))
-    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, std::max(need, P.bytes));
-  return prefill_run(q, w, k, q_offset, T_q, T_k, H, topk, out_idx, out_score,
-                     static_cast<uint8_t*>(workspace), P, true, true, static_cast<cudaStream_t>(stream));
+  // as many rows per launch as the workspace holds (all of them when it can)
+  const int64_t br = prefill_block_rows(T_q, T_k, H, topk, ws_bytes);
+  if (br < 1)
+    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes,
+                block_bytes(std::min<int64_t>(T_q, 256 / H), T_k, H, topk));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  for (int64_t r0 = 0; r0 < T_q; r0 += br) {
+    const int64_t n = std::min(br, T_q - r0);
+    const PrefillPlan P = plan_prefill(n, T_k, q_offset + r0, H, topk);
+    if (P.bytes > ws_bytes) return fail(DSA_EWORKSPACE, "internal: row block workspace too small");
+    rc = prefill_run(q + static_cast<size_t>(r0) * H * kD, w + static_cast<size_t>(r0) * H, k, q_offset + r0, n,
+                     T_k, H, topk, out_idx + static_cast<size_t>(r0) * topk, out_score + static_cast<size_t>(r0) * topk,
+                     ws, P, r0 == 0, r0 == 0, true, st);
+    if (rc != DSA_OK) return rc;
+  }
+  return DSA_OK;
 }
 
 size_t dsa_index_prefill_host_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
@@ -579,7 +757,7 @@ int dsa_index_prefill_host(const uint16_t* q, const float* w, const uint16_t* k,
     if ((rc = ck(cudaStreamWaitEvent(st, S->in[i], 0), "cudaStreamWaitEvent")) != DSA_OK) return rc;
     const PrefillPlan PB = plan_prefill(rows, T_k, q_offset + r0, H, topk);
     if (PB.bytes > P.ws_bytes) return fail(DSA_EWORKSPACE, "internal: block workspace too small");
-    if ((rc = prefill_run(dq, dw, dk, q_offset + r0, rows, T_k, H, topk, di, dsc, pws, PB, false, false, st)) !=
+    if ((rc = prefill_run(dq, dw, dk, q_offset + r0, rows, T_k, H, topk, di, dsc, pws, PB, false, false, false, st)) !=
         DSA_OK)
       return rc;
     if ((rc = ck(cudaEventRecord(S->comp[i], st), "cudaEventRecord")) != DSA_OK) return rc;
@@ -641,162 +819,101 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   auto at = [&](size_t off) { return ws + off; };
+  uint32_t* bypass = reinterpret_cast<uint32_t*>(at(P.off_ctl));
+  int32_t* row_flags = reinterpret_cast<int32_t*>(at(P.off_row_flags));
+  int32_t* refine_len = reinterpret_cast<int32_t*>(at(P.off_refine_len));
+  int32_t* surv_count = reinterpret_cast<int32_t*>(at(P.off_surv_count));
   cudaError_t e;
-  // zeroed state: status word, counters, seed bitmap, survivor counts
+  // zeroed state: status word, counters, control words, seed bitmap, survivor counts
   if ((e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  if ((e = cudaMemsetAsync(at(P.off_stats), 0, 8 * sizeof(unsigned long long), st)) != cudaSuccess)
-    return cuda_fail(e, "cudaMemsetAsync");
-  if ((e = cudaMemsetAsync(at(P.off_seed_bits), 0, P.mask_words * 4, st)) != cudaSuccess)
-    return cuda_fail(e, "cudaMemsetAsync");
-  if ((e = cudaMemsetAsync(at(P.off_surv_count), 0, T_q * 4, st)) != cudaSuccess)
+  if ((e = cudaMemsetAsync(at(P.off_stats), 0, 8 * sizeof(unsigned long long), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(bypass, 0, 8 * sizeof(uint32_t), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(at(P.off_seed_bits), 0, P.mask_words * 4, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(surv_count, 0, T_q * 4, st)) != cudaSuccess)
     return cuda_fail(e, "cudaMemsetAsync");
   prof_begin(st);
 
-  // 1. seeds: validate, mark, gather
+  // 1. seeds: validate, mark, gather; key norms for the screen
   SeedPrepParams sp0{seed_idx, n_seed, q_offset, k, reinterpret_cast<uint32_t*>(at(P.off_seed_bits)),
                      reinterpret_cast<uint16_t*>(at(P.off_k_seed)), err};
   if ((e = launch_seed_prep(sp0, st)) != cudaSuccess) return cuda_fail(e, "seed prep launch");
   prof_mark(st, "seed_prep");
-  // 2. seed scores with all heads; per row: sorted seed Top-k records and tau
-  CUtensorMap tq, tk, tks, tplan, tqrow;
-  if ((rc = make_tmap(&tq, q, T_q * H, P.seed.G * H)) != DSA_OK) return rc;
+  if ((e = launch_keynorm(k, T_k, reinterpret_cast<float*>(at(P.off_knorm)), st)) != cudaSuccess)
+    return cuda_fail(e, "keynorm launch");
+  prof_mark(st, "keynorm");
+  CUtensorMap tk, tqrow;
   if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
-  if ((rc = make_tmap(&tks, at(P.off_k_seed), n_seed, kTileKeys)) != DSA_OK) return rc;
-  if ((rc = make_tmap(&tplan, at(P.off_plan_q), T_q * kPlanRows, P.screen.G * kPlanRows)) != DSA_OK) return rc;
   if ((rc = make_tmap(&tqrow, q, T_q * H, H)) != DSA_OK) return rc;
-  {
-    ScoreParams s1{};
-    s1.mode = kModeGathered;
-    s1.topk = topk;
-    s1.lay = P.seed.lay;
-    s1.S = P.seed.S;
-    s1.n_groups = P.seed.n_groups;
-    s1.n_units = P.seed.n_units;
-    s1.q_offset = 0;
-    s1.T_q = T_q;
-    s1.T_k = n_seed;
-    s1.w = w;
-    s1.key_ids = seed_idx;
-    s1.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + P.seed.off_cand));
-    s1.meta = reinterpret_cast<int32_t*>(at(P.off_cand + P.seed.off_meta));
-    s1.err = err;
-    if ((e = launch_score(H, P.seed.G, P.seed.eg, tq, tks, s1, P.seed.grid, st)) != cudaSuccess)
-      return cuda_fail(e, "seed score launch");
-    prof_mark(st, "seed_score");
-    SelectParams s2{};
-    s2.mode = kModePrefill;
-    s2.G = P.seed.G;
-    s2.S = P.seed.S;
-    s2.topk = topk;
-    s2.lay = P.seed.lay;
-    s2.n_rows = T_q;
-    s2.cand = s1.cand;
-    s2.meta = s1.meta;
-    s2.out_rec = reinterpret_cast<uint64_t*>(at(P.off_seed_rec));
-    s2.rec_stride = P.rec_stride;
-    s2.out_kth = reinterpret_cast<float*>(at(P.off_tau));
-    s2.err = err;
-    if ((e = launch_select(s2, st)) != cudaSuccess) return cuda_fail(e, "seed select launch");
-    prof_mark(st, "seed_select");
+  // 2. the probe rows: seed scoring, plan, screen, compaction
+  if ((rc = pruned_rows(P, 0, 0, P.probe, q, w, q_offset, T_k, H, topk, seed_idx, n_seed, tk, ws, nullptr, st)) !=
+      DSA_OK)
+    return rc;
+  // 3. keep pruning the rest of the chunk, or mark it for the dense pass
+  if (P.probe < T_q) {
+    DecideParams dp{P.probe, T_q, q_offset, n_seed, surv_count, row_flags, refine_len, bypass};
+    if ((e = launch_decide(dp, st)) != cudaSuccess) return cuda_fail(e, "decide launch");
+    prof_mark(st, "decide");
+    if ((rc = pruned_rows(P, 1, P.probe, T_q - P.probe, q, w, q_offset, T_k, H, topk, seed_idx, n_seed, tk, ws,
+                          bypass, st)) != DSA_OK)
+      return rc;
   }
-  // 3. screening plan per row, key norms
-  {
-    PlanParams pp{q, w, reinterpret_cast<const uint16_t*>(at(P.off_k_seed)), n_seed, T_q,
-                  reinterpret_cast<const float*>(at(P.off_tau)), reinterpret_cast<uint16_t*>(at(P.off_plan_q)),
-                  reinterpret_cast<float*>(at(P.off_plan_s))};
-    if ((e = launch_plan(H, pp, st)) != cudaSuccess) return cuda_fail(e, "plan launch");
-    prof_mark(st, "plan");
-    if ((e = launch_keynorm(k, T_k, reinterpret_cast<float*>(at(P.off_knorm)), st)) != cudaSuccess)
-      return cuda_fail(e, "keynorm launch");
-    prof_mark(st, "keynorm");
-  }
-  // 4. screen every visible non-seed key: bound -> survivor bitmask
-  {
-    ScoreParams s3{};
-    s3.mode = kModePrefill;
-    s3.topk = topk;
-    s3.lay = P.screen.lay;
-    s3.S = P.screen.S;
-    s3.n_groups = P.screen.n_groups;
-    s3.n_units = P.screen.n_units;
-    s3.q_offset = q_offset;
-    s3.T_q = T_q;
-    s3.T_k = T_k;
-    s3.err = err;
-    s3.plan_s = reinterpret_cast<const float*>(at(P.off_plan_s));
-    s3.knorm = reinterpret_cast<const float*>(at(P.off_knorm));
-    s3.seed_bits = reinterpret_cast<const uint32_t*>(at(P.off_seed_bits));
-    s3.bitmask = reinterpret_cast<uint32_t*>(at(P.off_bitmask));
-    s3.mask_words = P.mask_words;
-    s3.surv_count = reinterpret_cast<int32_t*>(at(P.off_surv_count));
-    if ((e = launch_screen(tplan, tk, s3, P.screen.grid, st)) != cudaSuccess) return cuda_fail(e, "screen launch");
-    prof_mark(st, "screen");
-  }
-  // 5. compact survivors into id lists; flag rows for recovery
-  CompactParams cp{T_q, q_offset, topk, reinterpret_cast<const uint32_t*>(at(P.off_bitmask)), P.mask_words,
-                   reinterpret_cast<const int32_t*>(at(P.off_surv_count)), P.cap_row,
-                   reinterpret_cast<int32_t*>(at(P.off_surv_ids)), reinterpret_cast<int32_t*>(at(P.off_refine_len)),
-                   reinterpret_cast<int32_t*>(at(P.off_row_flags)), reinterpret_cast<const uint64_t*>(at(P.off_seed_rec)),
-                   P.rec_stride, reinterpret_cast<uint64_t*>(at(P.off_init_thr)), err};
-  if ((e = launch_compact(cp, st)) != cudaSuccess) return cuda_fail(e, "compact launch");
-  prof_mark(st, "compact");
-  // 6. refine survivors exactly (all heads), keeping records at or above the
+  // 4. refine survivors exactly (all heads), keeping records at or above the
   //    row's topk-th seed record, then the final exact Top-k over seed records
-  //    and refined candidates
-  {
-    uint8_t* rws = at(P.off_refine);
-    const DecodePlan& R = P.refine;
-    DecodePlanParams dp{};
-    dp.B = static_cast<int>(T_q);
-    dp.grid = R.grid;
-    dp.t_cap = P.cap_row;
-    dp.seq_len = reinterpret_cast<const int32_t*>(at(P.off_refine_len));
-    dp.seq_start = reinterpret_cast<int64_t*>(rws + R.off_seq_start);
-    dp.unit_tab = reinterpret_cast<int32_t*>(rws + R.off_unit_tab);
-    dp.cta_ubeg = reinterpret_cast<int32_t*>(rws + R.off_cta_ubeg);
-    dp.seq_ubeg = reinterpret_cast<int32_t*>(rws + R.off_seq_ubeg);
-    dp.seq_ucnt = reinterpret_cast<int32_t*>(rws + R.off_seq_ucnt);
-    dp.err = err;
-    if ((e = launch_decode_plan(dp, st)) != cudaSuccess) return cuda_fail(e, "refine plan launch");
-    ScoreParams s4{};
-    s4.mode = kModeRefine;
-    s4.topk = topk;
-    s4.lay = R.lay;
-    s4.S = 1;
-    s4.T_k = T_k;
-    s4.w = w;
-    s4.seq_len = dp.seq_len;
-    s4.unit_tab = dp.unit_tab;
-    s4.cta_ubeg = dp.cta_ubeg;
-    s4.cand = reinterpret_cast<uint64_t*>(rws + R.off_cand);
-    s4.meta = reinterpret_cast<int32_t*>(rws + R.off_meta);
-    s4.err = err;
-    s4.surv_ids = reinterpret_cast<const int32_t*>(at(P.off_surv_ids));
-    s4.surv_stride = P.cap_row;
-    s4.k_gather = k;
-    s4.init_thr = reinterpret_cast<const uint64_t*>(at(P.off_init_thr));
-    if ((e = launch_score(H, 1, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
-    prof_mark(st, "refine");
-    SelectParams s5{};
-    s5.mode = kModeDecode;
-    s5.G = 1;
-    s5.S = 1;
-    s5.topk = topk;
-    s5.lay = R.lay;
-    s5.n_rows = T_q;
-    s5.cand = s4.cand;
-    s5.meta = s4.meta;
-    s5.seq_ubeg = dp.seq_ubeg;
-    s5.seq_ucnt = dp.seq_ucnt;
-    s5.extra_rec = reinterpret_cast<const uint64_t*>(at(P.off_seed_rec));
-    s5.rec_stride = P.rec_stride;
-    s5.out_idx = out_idx;
-    s5.out_score = out_score;
-    s5.err = err;
-    if ((e = launch_select(s5, st)) != cudaSuccess) return cuda_fail(e, "final select launch");
-    prof_mark(st, "final_select");
-  }
-  // 7. exact recovery: flagged rows are recomputed by the dense path
+  //    and refined candidates of the rows that came out of the screen exact
+  uint8_t* rws = at(P.off_refine);
+  const DecodePlan& R = P.refine;
+  DecodePlanParams dq{};
+  dq.B = static_cast<int>(T_q);
+  dq.grid = R.grid;
+  dq.t_cap = P.cap_row;
+  dq.seq_len = refine_len;
+  dq.seq_start = reinterpret_cast<int64_t*>(rws + R.off_seq_start);
+  dq.unit_tab = reinterpret_cast<int32_t*>(rws + R.off_unit_tab);
+  dq.cta_ubeg = reinterpret_cast<int32_t*>(rws + R.off_cta_ubeg);
+  dq.seq_ubeg = reinterpret_cast<int32_t*>(rws + R.off_seq_ubeg);
+  dq.seq_ucnt = reinterpret_cast<int32_t*>(rws + R.off_seq_ucnt);
+  dq.err = err;
+  if ((e = launch_decode_plan(dq, st)) != cudaSuccess) return cuda_fail(e, "refine plan launch");
+  ScoreParams s4{};
+  s4.mode = kModeRefine;
+  s4.topk = topk;
+  s4.lay = R.lay;
+  s4.S = 1;
+  s4.T_k = T_k;
+  s4.w = w;
+  s4.seq_len = dq.seq_len;
+  s4.unit_tab = dq.unit_tab;
+  s4.cta_ubeg = dq.cta_ubeg;
+  s4.cand = reinterpret_cast<uint64_t*>(rws + R.off_cand);
+  s4.meta = reinterpret_cast<int32_t*>(rws + R.off_meta);
+  s4.err = err;
+  s4.surv_ids = reinterpret_cast<const int32_t*>(at(P.off_surv_ids));
+  s4.surv_stride = P.cap_row;
+  s4.k_gather = k;
+  s4.init_thr = reinterpret_cast<const uint64_t*>(at(P.off_init_thr));
+  if ((e = launch_score(H, 1, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
+  prof_mark(st, "refine");
+  SelectParams s5{};
+  s5.mode = kModeDecode;
+  s5.G = 1;
+  s5.S = 1;
+  s5.topk = topk;
+  s5.lay = R.lay;
+  s5.n_rows = T_q;
+  s5.cand = s4.cand;
+  s5.meta = s4.meta;
+  s5.seq_ubeg = dq.seq_ubeg;
+  s5.seq_ucnt = dq.seq_ucnt;
+  s5.extra_rec = reinterpret_cast<const uint64_t*>(at(P.off_seed_rec));
+  s5.rec_stride = P.rec_stride;
+  s5.row_flags = row_flags;
+  s5.skip_flagged = 1;
+  s5.out_idx = out_idx;
+  s5.out_score = out_score;
+  s5.err = err;
+  if ((e = launch_select(s5, st)) != cudaSuccess) return cuda_fail(e, "final select launch");
+  prof_mark(st, "final_select");
+  // 5. exact dense pass over every flagged row (overflow, bad seeds, bypass)
   {
     ScoreParams s6{};
     s6.mode = kModePrefill;
@@ -812,11 +929,12 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     s6.cand = reinterpret_cast<uint64_t*>(at(P.off_cand + P.dense.off_cand));
     s6.meta = reinterpret_cast<int32_t*>(at(P.off_cand + P.dense.off_meta));
     s6.err = err;
-    s6.row_flags = reinterpret_cast<const int32_t*>(at(P.off_row_flags));
+    s6.row_flags = row_flags;
     CUtensorMap tqd;
     if ((rc = make_tmap(&tqd, q, T_q * H, P.dense.G * H)) != DSA_OK) return rc;
     if ((e = launch_score(H, P.dense.G, P.dense.eg, tqd, tk, s6, P.dense.grid, st)) != cudaSuccess)
       return cuda_fail(e, "recovery launch");
+    prof_mark(st, "dense_pass");
     SelectParams s7{};
     s7.mode = kModePrefill;
     s7.G = P.dense.G;
@@ -828,34 +946,54 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     s7.meta = s6.meta;
     s7.out_idx = out_idx;
     s7.out_score = out_score;
-    s7.row_flags = s6.row_flags;
+    s7.row_flags = row_flags;
     s7.err = err;
     if ((e = launch_select(s7, st)) != cudaSuccess) return cuda_fail(e, "recovery select launch");
-    prof_mark(st, "recovery");
+    prof_mark(st, "dense_select");
   }
   if (stats) {
     unsigned long long* cnt = reinterpret_cast<unsigned long long*>(at(P.off_stats));
-    if ((e = launch_stats(reinterpret_cast<const int32_t*>(at(P.off_surv_count)),
-                          reinterpret_cast<const int32_t*>(at(P.off_refine_len)),
-                          reinterpret_cast<const int32_t*>(at(P.off_row_flags)), T_q, cnt, st)) != cudaSuccess)
-      return cuda_fail(e, "stats launch");
+    StatsParams sp{T_q, q_offset, n_seed, topk, R.lay, surv_count, refine_len, row_flags, s4.meta,
+                   dq.seq_ubeg, dq.seq_ucnt, cnt};
+    if ((e = launch_stats(sp, st)) != cudaSuccess) return cuda_fail(e, "stats launch");
     unsigned long long h[8] = {};
     uint32_t status = 0;
     if ((e = cudaMemcpyAsync(h, cnt, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
         (e = cudaMemcpyAsync(&status, err, 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
         (e = cudaStreamSynchronize(st)) != cudaSuccess)
       return cuda_fail(e, "reading the pruned-path counters");
-    // screened: every visible key of every row except the row's seeds
-    const int64_t vis = (2 * q_offset + T_q + 1) * T_q / 2;
-    stats->screened_pairs = vis - T_q * static_cast<int64_t>(n_seed);
     stats->survivor_pairs = static_cast<int64_t>(h[0]);
     stats->refined_pairs = static_cast<int64_t>(h[1]);
     stats->recovered_rows = static_cast<int64_t>(h[2]);
-    stats->records = T_q * static_cast<int64_t>(topk) + static_cast<int64_t>(h[1]);
+    stats->bypassed_rows = static_cast<int64_t>(h[3]);
+    stats->screened_pairs = static_cast<int64_t>(h[4]);
+    stats->records = static_cast<int64_t>(h[5]);
     if (status & kErrSeed) return fail(DSA_ESEED, "a seed was out of range or repeated; the rows were recomputed densely");
     if (status & kErrTimeout) return fail(DSA_EDEVICE, "a device-side wait gave up (status 0x%x)", status);
     if (status & kErrNonFinite) return fail(DSA_EDEVICE, "a visible pair scored inf or NaN (non-finite input)");
   }
+  return DSA_OK;
+}
+
+int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_q, int64_t T_k, int64_t q_offset, int H,
+                                       int d, int topk, int n_seed, uint32_t* mask, float* tau, int32_t* row_state,
+                                       void* stream) {
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (T_q < 1 || T_k < 1 || q_offset < 0 || q_offset + T_q > T_k || n_seed < 1)
+    return fail(DSA_EINVAL, "need T_q >= 1, T_k >= 1, 0 <= q_offset, q_offset + T_q <= T_k, n_seed >= 1");
+  if (!workspace || !mask || !tau || !row_state) return fail(DSA_EINVAL, "null pointer argument");
+  const PrunedPlan P = plan_pruned(T_q, T_k, q_offset, H, topk, n_seed);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(mask, ws + P.off_bitmask, static_cast<size_t>(T_q) * P.mask_words * 4,
+                           cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(tau, ws + P.off_tau, static_cast<size_t>(T_q) * 4, cudaMemcpyDeviceToDevice, st)) !=
+          cudaSuccess ||
+      (e = cudaMemcpyAsync(row_state, ws + P.off_row_flags, static_cast<size_t>(T_q) * 4, cudaMemcpyDeviceToDevice,
+                           st)) != cudaSuccess)
+    return cuda_fail(e, "copying the screen's survivor mask");
   return DSA_OK;
 }
 
@@ -881,6 +1019,18 @@ int dsa_index_decode_noalloc(const uint16_t* q, const float* w, const uint16_t* 
   if ((rc = noalloc_scratch(&ws)) != DSA_OK) return rc;
   return decode_run(q, w, k_cache, seq_len, B, t_cap, H, topk, out_idx, out_score,
                     static_cast<uint8_t*>(ws), P, false, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_index_decode_noalloc_status(uint32_t* status, void* stream) {
+  if (!status) return fail(DSA_EINVAL, "null pointer argument");
+  void* ws = nullptr;
+  int rc = noalloc_scratch(&ws);
+  if (rc != DSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(status, ws, 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the static scratch's device status word");
+  return DSA_OK;
 }
 
 int dsa_profile_enable(int on) {

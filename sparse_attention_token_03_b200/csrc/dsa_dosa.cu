@@ -8,6 +8,8 @@
 //                       bound, folded positive / negative auxiliary rows and
 //                       the scalars of the screening bound
 //   compact_kernel      survivor bitmask -> ascending survivor id list per row
+//   decide_kernel       after the probe rows: keep pruning or send the rest of
+//                       the chunk to the dense path
 //   stats_kernel        counters for the dsa_stats struct
 //
 // The screening MMA and the exact refine are variants of the fused score
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
   __shared__ float wal[4][R];   // per-warp alpha partials
   __shared__ float wbe[4];      // per-warp beta partials
 
+  if (p.skip && *p.skip) return;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint16_t* qrow = p.q + static_cast<size_t>(t) * H * kD;
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
 __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
   __shared__ int s_scan[256 / 32];
   __shared__ int s_base;
+  if (p.skip && *p.skip) return;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int count = p.surv_count[t];
@@ -360,13 +364,13 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
   if (tid == 0) p.init_thr[t] = p.seed_rec[static_cast<size_t>(t) * p.rec_stride + p.topk - 1];
   if (bad_seed || count > p.cap_row) {
     if (tid == 0) {
-      p.row_flags[t] = 1;
+      p.row_flags[t] = bad_seed ? kRowBadSeed : kRowOverflow;
       p.refine_len[t] = 0;
     }
     return;
   }
   if (tid == 0) {
-    p.row_flags[t] = 0;
+    p.row_flags[t] = kRowRefined;
     p.refine_len[t] = count;
     s_base = 0;
   }
@@ -403,19 +407,103 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
   }
 }
 
-// Sums for dsa_stats (one CTA): survivor pairs, refined pairs, flagged rows.
-__global__ void __launch_bounds__(256) stats_kernel(const int32_t* surv_count, const int32_t* refine_len,
-                                                     const int32_t* row_flags, int64_t T_q,
-                                                     unsigned long long* out) {
-  unsigned long long a = 0, b = 0, c = 0;
-  for (int64_t t = threadIdx.x; t < T_q; t += blockDim.x) {
-    a += static_cast<unsigned long long>(surv_count[t]);
-    b += static_cast<unsigned long long>(refine_len[t]);
-    c += row_flags[t] ? 1ull : 0ull;
+// ---------------------------------------------------------------------------
+// Probe decision (one CTA of 256 threads).  The probe rows went through the
+// whole pruned path; from them, estimate the pruned cost of a row relative to
+// its dense cost:
+//   kScreenCost                       screening every visible key
+//   + kSeedCost * n_seed / v          scoring the seeds with all heads
+//   + kPlanPairs / v                  the per-row plan
+//   + overflow fraction               rows recomputed densely
+//   + kRefineCost * refined / pairs   exact refine of the survivors
+// (v = mean visible keys of a probe row).  The constants are the measured
+// per-pair costs of these kernels on B200 relative to the dense kernel's
+// (128K and 1M chunks).  When the estimate reaches 1 the remaining rows skip
+// the pruned path and are marked for the dense pass.
+// ---------------------------------------------------------------------------
+constexpr float kScreenCost = 0.6f;
+constexpr float kSeedCost = 1.6f;
+constexpr float kPlanPairs = 15000.0f;
+constexpr float kRefineCost = 10.0f;
+
+__global__ void __launch_bounds__(256) decide_kernel(const DecideParams p) {
+  __shared__ float s_red[3][8];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  float over = 0.0f, refined = 0.0f, vis = 0.0f;
+  for (int64_t t = tid; t < p.probe_rows; t += 256) {
+    const bool ok = p.row_flags[t] == kRowRefined;
+    over += ok ? 0.0f : 1.0f;
+    refined += ok ? static_cast<float>(p.surv_count[t]) : 0.0f;
+    vis += static_cast<float>(p.q_offset + t + 1);
   }
-  atomicAdd(&out[0], a);
-  atomicAdd(&out[1], b);
-  atomicAdd(&out[2], c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    over += __shfl_xor_sync(0xFFFFFFFFu, over, o);
+    refined += __shfl_xor_sync(0xFFFFFFFFu, refined, o);
+    vis += __shfl_xor_sync(0xFFFFFFFFu, vis, o);
+  }
+  if (lane == 0) {
+    s_red[0][wid] = over;
+    s_red[1][wid] = refined;
+    s_red[2][wid] = vis;
+  }
+  __syncthreads();
+  __shared__ int s_bypass;
+  if (tid == 0) {
+    float o = 0.0f, r = 0.0f, v = 0.0f;
+    for (int i = 0; i < 8; ++i) {
+      o += s_red[0][i];
+      r += s_red[1][i];
+      v += s_red[2][i];
+    }
+    const float n = static_cast<float>(p.probe_rows);
+    const float vbar = v / n;
+    const float est = kScreenCost + kSeedCost * static_cast<float>(p.n_seed) / vbar + kPlanPairs / vbar + o / n +
+                      kRefineCost * r / v;
+    s_bypass = est >= 1.0f ? 1 : 0;
+    *p.bypass = static_cast<uint32_t>(s_bypass);
+  }
+  __syncthreads();
+  if (!s_bypass) return;
+  for (int64_t t = p.probe_rows + tid; t < p.T_q; t += 256) {
+    p.row_flags[t] = kRowBypassed;
+    p.refine_len[t] = 0;
+  }
+}
+
+// Sums for dsa_stats (one CTA): out[0] survivor pairs, [1] refined pairs,
+// [2] rows recovered after screening, [3] bypassed rows, [4] screened pairs,
+// [5] records the final selection read (seed Top-k + refined candidates of
+// the rows it finished).
+__global__ void __launch_bounds__(256) stats_kernel(const StatsParams p) {
+  unsigned long long a = 0, b = 0, c = 0, by = 0, sc = 0, rec = 0;
+  for (int64_t t = threadIdx.x; t < p.T_q; t += blockDim.x) {
+    const int32_t f = p.row_flags[t];
+    if (f == kRowBypassed) {
+      ++by;
+      continue;
+    }
+    a += static_cast<unsigned long long>(p.surv_count[t]);
+    b += static_cast<unsigned long long>(p.refine_len[t]);
+    sc += static_cast<unsigned long long>(p.q_offset + t + 1 - p.n_seed);
+    if (f != kRowRefined) {
+      ++c;
+      continue;
+    }
+    rec += static_cast<unsigned long long>(p.topk);
+    const int u0 = p.seq_ubeg[t], nu = p.seq_ucnt[t];
+    for (int u = u0; u < u0 + nu; ++u) {
+      const int32_t* m = p.meta + static_cast<size_t>(u) * kMetaInts;
+      rec += static_cast<unsigned long long>(min(max(m[1], 0), p.lay.keep_cap));
+      for (int r = 0; r < 4; ++r) rec += static_cast<unsigned long long>(min(max(m[2 + r], 0), p.lay.app_cap));
+    }
+  }
+  atomicAdd(&p.out[0], a);
+  atomicAdd(&p.out[1], b);
+  atomicAdd(&p.out[2], c);
+  atomicAdd(&p.out[3], by);
+  atomicAdd(&p.out[4], sc);
+  atomicAdd(&p.out[5], rec);
 }
 
 cudaError_t launch_seed_prep(const SeedPrepParams& p, cudaStream_t st) {
@@ -444,9 +532,13 @@ cudaError_t launch_compact(const CompactParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_stats(const int32_t* surv_count, const int32_t* refine_len, const int32_t* row_flags,
-                         int64_t T_q, unsigned long long* out, cudaStream_t st) {
-  stats_kernel<<<1, 256, 0, st>>>(surv_count, refine_len, row_flags, T_q, out);
+cudaError_t launch_decide(const DecideParams& p, cudaStream_t st) {
+  decide_kernel<<<1, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats(const StatsParams& p, cudaStream_t st) {
+  stats_kernel<<<1, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@ struct PlanParams {
   const float* tau;        // [T_q] topk-th seed score per row
   uint16_t* plan_q;        // [T_q][kPlanRows][128]
   float* plan_s;           // [T_q][kPlanScalars]
+  const uint32_t* skip;    // optional: when *skip != 0 the launch does nothing
 };
 
 struct CompactParams {
@@ -44,13 +45,53 @@ struct CompactParams {
   int rec_stride;
   uint64_t* init_thr;       // [T_q]
   const uint32_t* err;
+  const uint32_t* skip;     // optional: when *skip != 0 the launch does nothing
+};
+
+// Row states of the pruned path (row_flags): every non-zero state is
+// recomputed by the dense recovery pass.
+enum : int32_t {
+  kRowRefined = 0,    // screened; survivors refined exactly
+  kRowOverflow = 1,   // screened; survivors exceeded the row's list
+  kRowBypassed = 2,   // not screened: the probe sent the chunk to the dense path
+  kRowBadSeed = 3,    // the seed list failed validation
+};
+
+// Probe decision: after the first rows of a chunk went through the pruned
+// path, estimate the pruned cost of the chunk relative to the dense cost and
+// set *bypass when pruning would not pay.
+struct DecideParams {
+  int64_t probe_rows;
+  int64_t T_q;
+  int64_t q_offset;
+  int n_seed;
+  const int32_t* surv_count;  // [T_q]
+  int32_t* row_flags;         // [T_q]
+  int32_t* refine_len;        // [T_q]
+  uint32_t* bypass;           // control word
+};
+
+// Counters of dsa_stats, summed on the device.
+struct StatsParams {
+  int64_t T_q;
+  int64_t q_offset;
+  int n_seed;
+  int topk;
+  CandLayout lay;            // refine candidate layout
+  const int32_t* surv_count;
+  const int32_t* refine_len;
+  const int32_t* row_flags;
+  const int32_t* meta;       // refine candidate meta, [unit][kMetaInts]
+  const int32_t* seq_ubeg;   // refine units per row
+  const int32_t* seq_ucnt;
+  unsigned long long* out;   // [8]
 };
 
 cudaError_t launch_seed_prep(const SeedPrepParams& p, cudaStream_t st);
 cudaError_t launch_keynorm(const uint16_t* k, int64_t T_k, float* knorm, cudaStream_t st);
 cudaError_t launch_plan(int H, const PlanParams& p, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams& p, cudaStream_t st);
-cudaError_t launch_stats(const int32_t* surv_count, const int32_t* refine_len, const int32_t* row_flags,
-                         int64_t T_q, unsigned long long* out, cudaStream_t st);
+cudaError_t launch_decide(const DecideParams& p, cudaStream_t st);
+cudaError_t launch_stats(const StatsParams& p, cudaStream_t st);
 
 }  // namespace dsa

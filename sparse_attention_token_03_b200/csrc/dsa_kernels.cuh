@@ -7,7 +7,7 @@
 // compaction kept) and four append regions of app_cap records, one per
 // epilogue warp (TMEM lane quarter), so that admissions need no atomics.
 // Meta per (slot, query): kMetaInts ints = {active half, base count, four
-// append counts}.  Records are 64-bit (score code << 32 | ~key): unsigned
+// append counts, admission threshold record (low word, high word)}.  Records are 64-bit (score code << 32 | ~key): unsigned
 // order is the selection order, and 0 is never a record.
 #pragma once
 
@@ -135,6 +135,12 @@ struct ScoreParams {
   int32_t* meta;
   uint32_t* err;
   const int32_t* row_flags; // prefill: when set, groups without a flagged row do nothing
+  const uint32_t* skip;     // optional: when *skip != 0 the launch does nothing
+  // failure injection for tests (dsa_test_inject_wait_timeout): when set, the
+  // producer issues no loads, so the MMA warp's first wait runs out after
+  // wait_ns and the launch unwinds with the timeout bit
+  int stall_loads;
+  uint64_t wait_ns;         // limit of the pipeline waits (0: kWaitTimeoutNs)
   // refine: survivor key ids per row (stride surv_stride), the key matrix they
   // index, and an initial admission threshold record per row
   const int32_t* surv_ids;
@@ -165,6 +171,8 @@ struct SelectParams {
   const uint64_t* extra_rec;  // optional [n_rows][rec_stride] extra records (0 = none) merged per row
   int rec_stride;             // row stride of extra_rec / out_rec (>= topk, even)
   const int32_t* row_flags;   // optional: only rows with a non-zero flag are written
+  int skip_flagged;           // with row_flags: write only the rows whose flag is zero instead
+  const uint32_t* skip;       // optional: when *skip != 0 the launch does nothing
   int32_t* out_idx;         // [n_rows][topk] (may be null when out_rec is set)
   float* out_score;         // [n_rows][topk]
   uint64_t* out_rec;        // optional [n_rows][rec_stride] records (sorted, 0-padded)
@@ -217,6 +225,10 @@ struct ScoreSmem {
   // dynamic smem request: layout + slack to align the base to 1024 bytes
   __host__ __device__ constexpr uint32_t request() const { return bytes() + 1024u; }
 };
+
+// Host side of the failure injection: moves a pending one-shot injection of
+// the calling thread into the launch's parameters (dsa_api.cu).
+void take_wait_injection(ScoreParams& p);
 
 // Launchers (defined in the .cu files).
 cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,

@@ -32,6 +32,8 @@
 // to a value with at least k buffered records at or above it, so any later
 // key below it (records order by score, then smaller key first) can never
 // enter the Top-k.
+#include <atomic>
+
 #include "dsa_kernels.cuh"
 #include "dsa_ptx.cuh"
 
@@ -276,6 +278,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
   static_assert(G % EG == 0, "queries must split evenly over the epilogue warpgroups");
 
+  if (p.skip && *p.skip) return;  // whole launch disabled by an earlier kernel (uniform)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -324,11 +327,12 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   const uint32_t tmem_base = *s_tmem;
 
   const int u_begin = cta_unit_begin(p), u_end = cta_unit_end(p), u_step = cta_unit_step(p);
+  const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitTimeoutNs;  // pipeline waits
 
   if (warp < score_epi_warp0(EG)) {
    // one setmaxnreg for the whole control warpgroup
    if constexpr (EG >= 2) regs_dec<regs_ctl(EG)>();
-   if (warp == 0 && p.mode == kModeRefine) {
+   if (warp == 0 && p.mode == kModeRefine && !p.stall_loads) {
     // ------------------------------------------------ producer (gathered keys)
     // Survivor keys are gathered row by row with 16-byte cp.async into the
     // 128B-swizzled layout the MMA reads.  A stage is signalled LAG tiles
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       if (U.tile_hi <= U.tile_lo) continue;
       drain();  // the MMA must see this unit's predecessor complete before the query tile changes
       if (lane == 0) {
-        ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err);
+        ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err, wlim);
         if (ok) {
           mbar_arrive_expect_tx(bar_q_full, L.q_bytes());
           tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       const int64_t n = U.vis_base;
       for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
         const int s = kt % NS;
-        if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err))) break;
+        if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err, wlim))) break;
         const uint32_t stage = sK + s * L.k_stage();
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     drain();
    } else if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !p.stall_loads) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       uint32_t kt = 0, qi = 0;
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       for (int u = u_begin; ok && u < u_end; u += u_step) {
         const Unit U = unit_geometry<G>(p, u, H);
         if (U.tile_hi <= U.tile_lo) continue;
-        if (!(ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err))) break;
+        if (!(ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err, wlim))) break;
         mbar_arrive_expect_tx(bar_q_full, L.q_bytes());
         tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
         tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         }
         for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
           const int s = kt % NS;
-          if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err))) break;
+          if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err, wlim))) break;
           mbar_arrive_expect_tx(bar_k_full(s), L.k_stage());
           const int32_t krow = static_cast<int32_t>(U.k_row + t * kTileKeys);
           tma_load_2d(sK + s * L.k_stage(), &tmap_k, 0, krow, bar_k_full(s));
@@ -434,13 +438,13 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       for (int u = u_begin; ok && u < u_end; u += u_step) {
         const Unit U = unit_geometry<G>(p, u, H);
         if (U.tile_hi <= U.tile_lo) continue;
-        if (!(ok = mbar_wait(bar_q_full, qi & 1, s_abort, p.err))) break;
+        if (!(ok = mbar_wait(bar_q_full, qi & 1, s_abort, p.err, wlim))) break;
         ++qi;
         for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
           const int s = kt % NS;
           const int a = at & 1;
-          if (!(ok = mbar_wait(bar_k_full(s), (kt / NS) & 1, s_abort, p.err))) break;
-          if (!(ok = mbar_wait(bar_acc_empty(a), ((at >> 1) & 1) ^ 1, s_abort, p.err))) break;
+          if (!(ok = mbar_wait(bar_k_full(s), (kt / NS) & 1, s_abort, p.err, wlim))) break;
+          if (!(ok = mbar_wait(bar_acc_empty(a), ((at >> 1) & 1) ^ 1, s_abort, p.err, wlim))) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + a * ACC_COLS;
           const uint32_t a_base = sK + s * L.k_stage();
@@ -511,7 +515,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       for (int i = 0; i < GQ; ++i) surv[i] = 0;
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
-        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
+        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err, wlim))) break;
         tc_fence_after();
         const int64_t key_local = t * kTileKeys + row_in_tile;
         const bool in_range = key_local < p.T_k;
@@ -647,7 +651,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       bool nonfinite = false;  // a visible pair scored inf or NaN (reported at the unit's end)
       for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
         const int a = at & 1;
-        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err))) break;
+        if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err, wlim))) break;
         tc_fence_after();
         const int64_t key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
@@ -738,7 +742,9 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           // topk of them in bins >= B, a later key whose score code lies below
           // bin B is beaten by topk records and can never be selected.
           int kept_above = 0;
-          if (total >= p.topk && (full || total - s_upd[qq] >= 256)) {
+          // (at the unit's last tile always: the final threshold goes to the
+          // unit's meta, where the final selection filters by it)
+          if (total >= p.topk && (full || total - s_upd[qq] >= 256 || t + 1 == U.tile_hi)) {
             epi_find_bucket(qh, kHistBins, 0, p.topk, etid, s_misc + 4, s_misc + 1, bar);
             const uint64_t t_new = static_cast<uint64_t>(hist_edge(static_cast<uint32_t>(s_misc[1]))) << 32;
             kept_above = s_misc[2] + s_misc[3];
@@ -841,6 +847,10 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         m[1] = s_count[qq];
 #pragma unroll
         for (int w2 = 0; w2 < 4; ++w2) m[2 + w2] = s_wcnt[qq * 4 + w2];
+        // the unit's admission threshold: at least topk of its buffered
+        // records are >= it once it is above the initial one
+        m[6] = static_cast<int32_t>(static_cast<uint32_t>(s_thr[qq]));
+        m[7] = static_cast<int32_t>(static_cast<uint32_t>(s_thr[qq] >> 32));
       }
     }
   }
@@ -864,8 +874,10 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
   auto kern = score_topk_kernel<H, G, NS, EG, EPI>;
   int dev = 0;
   cudaGetDevice(&dev);
-  static bool configured[64] = {};
-  if (dev < 64 && !configured[dev]) {
+  // per (kernel instance, device); racing host threads only repeat the
+  // idempotent attribute calls
+  static std::atomic<bool> configured[64];
+  if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L.request()));
     if (e != cudaSuccess) return e;
@@ -877,14 +889,16 @@ static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
       if (e != cudaSuccess) return e;
       if (fa.numRegs != static_cast<int>(regs_launch(EG))) return cudaErrorInvalidConfiguration;
     }
-    configured[dev] = true;
+    if (dev >= 0 && dev < 64) configured[dev].store(true, std::memory_order_release);
   }
   kern<<<grid, score_threads(EG), L.request(), stream>>>(tq, tk, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const ScoreParams& p, int grid, cudaStream_t stream) {
+                         const ScoreParams& p0, int grid, cudaStream_t stream) {
+  ScoreParams p = p0;
+  take_wait_injection(p);
   if (H == 64 && G == 4 && eg == 4) return launch_score_t<64, 4, 4, 4>(tq, tk, p, grid, stream);
   if (H == 64 && G == 4 && eg == 2) return launch_score_t<64, 4, 4, 2>(tq, tk, p, grid, stream);
   if (H == 32 && G == 8 && eg == 4) return launch_score_t<32, 8, 3, 4>(tq, tk, p, grid, stream);
@@ -897,8 +911,10 @@ cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tq, const CUte
 // Screening: 16 plan rows per query, kScreenQueries = 8 queries per MMA
 // (N = 128), four per epilogue thread so that their bound coefficients fit in
 // registers.
-cudaError_t launch_screen(const CUtensorMap& tplan, const CUtensorMap& tk, const ScoreParams& p,
+cudaError_t launch_screen(const CUtensorMap& tplan, const CUtensorMap& tk, const ScoreParams& p0,
                           int grid, cudaStream_t stream) {
+  ScoreParams p = p0;
+  take_wait_injection(p);
   return launch_score_t<kPlanRows, kScreenQueries, 5, 2, kEpiScreen>(tplan, tk, p, grid, stream);
 }
 

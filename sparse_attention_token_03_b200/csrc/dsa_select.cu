@@ -1,17 +1,29 @@
 // Final exact Top-k over candidate records, and the decode work planner.
 //
-// select_topk_kernel: one CTA per output row.  It merges the row's candidate
-// buffers (one per key split), finds the m-th largest record exactly
-// (m = min(k, candidates); 11-bit radix passes over the 64-bit records,
-// top digits first, stopping as soon as the selected prefix holds exactly
-// the records still needed), gathers the m winners into shared memory and
-// bitonic-sorts them (score descending, then key ascending: the order of the
-// records as unsigned integers).  Rows are padded with key -1 / score -inf
-// past m ("DeepSeek DSA FLOPs", selected pair count: a row keeps min(k, visible)).
+// select_topk_kernel: one CTA of 256 threads per output row.  It merges the
+// row's candidate buffers (one per key split, plus an optional segment of
+// extra records) into the row's m = min(k, candidates) largest records,
+// sorted by score descending, then key ascending (the order of the records
+// as unsigned integers), and pads the row with key -1 / score -inf past m
+// ("DeepSeek DSA FLOPs", selected pair count: a row keeps min(k, visible)).
+//
+// Every candidate buffer carries its unit's final admission threshold: at
+// least k of the unit's records are at or above it, so no record below the
+// largest of these thresholds can be selected.  One coalesced pass over the
+// row's buffers stages only the records at or above it (usually a little
+// more than k) in shared memory; a counting pass over a digit that is linear
+// in the score (1024 buckets between the staged minimum and maximum) finds
+// the bucket holding the m-th record, the records from that bucket up are
+// scattered into bucket order, and a rank count inside each bucket places
+// every winner; the row is written in order.  Rows with more records than the
+// staging buffer holds, or whose winners crowd one bucket, take an exact
+// radix select (10-bit digits) and a bitonic sort instead.  Shared memory
+// stays at about 50 KB so that four rows run on each SM at once.
 //
 // decode_plan_kernel: splits the flattened (sequence, key tile) space of a
 // batched decode evenly over the persistent score CTAs and emits the unit
 // table (one unit per CTA x sequence overlap).
+#include <atomic>
 #include <cfloat>
 
 #include "dsa_kernels.cuh"
@@ -21,14 +33,13 @@ namespace dsa {
 
 namespace {
 
-constexpr int kStageRecs = 7680;  // candidates of a row staged in shared memory (60 KB)
-constexpr int kWinCap = 4096;     // records in the boundary bucket and above it (32 KB)
-constexpr int kRankMax = 256;     // largest bucket ranked by counting
-constexpr int kBatch = 4;         // staged records per thread per step of a pass
-
-__device__ __forceinline__ void hist_add_blk(uint32_t* hist, bool valid, uint32_t digit) {
-  if (valid) atomicAdd(&hist[digit], 1u);
-}
+constexpr int kSelBins = 1024;   // buckets of the counting select and radix digits (10 bits)
+constexpr int kSelStage = 3072;  // records at or above the row threshold staged in shared memory
+constexpr int kSelSegs = 320;    // candidate segments of a row tabulated in shared memory
+constexpr int kRankMax = 256;    // largest bucket ranked by counting
+constexpr int kBatch = 4;        // records per thread per step of a pass
+constexpr size_t kSelectSmem = (kSelStage + kMaxTopk) * sizeof(uint64_t);  // staging + output (dynamic)
+static_assert(kSelStage >= kMaxTopk, "the sort exchange reuses the staging buffer");
 
 // Block-wide: largest bucket B with above + sum_{d >= B} hist[d] >= need.
 // Writes {B, above + sum_{d > B} hist[d], hist[B]} to res.
@@ -140,42 +151,49 @@ __device__ __forceinline__ void sort2048_desc(uint64_t (&v)[8], uint64_t* s_x) {
   }
 }
 
+// Warp-aggregated append of the kept records of one step into s_rec
+// (positions past cap are counted but not written).
+__device__ __forceinline__ void stage_append(bool keep, uint64_t r, uint64_t* s_rec, int cap, int* s_n, int lane) {
+  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+  if (bal == 0u) return;
+  int pos = 0;
+  if (lane == 0) pos = atomicAdd(s_n, __popc(bal));
+  pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+  const int at = pos + __popc(bal & lanemask_lt());
+  if (keep && at < cap) s_rec[at] = r;
+}
+
 }  // namespace
 
-// One CTA of 256 threads per output row.
-//
-// Staged rows (the usual case) take one counting pass: a 2048-bucket digit
-// of each record that never decreases along the record order (linear in the
-// score over the row's score range), a descending prefix scan of the bucket
-// counts, which also finds the bucket holding the m-th record, a scatter of
-// every record in that bucket or above it into bucket order, and a rank
-// count inside each bucket that gives each winner its final position (the
-// row's output is then written in order).  Rows whose candidates do not fit the staging buffer, or whose
-// records crowd more than kRankMax into one bucket, take the radix-select +
-// bitonic-sort path instead.
 template <int NT>
-__global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p) {
   static_assert(NT == 256, "the sort layout assumes 256 threads x 8 records");
   extern __shared__ __align__(16) uint64_t s_dyn[];
-  uint64_t* s_rec = s_dyn;               // [kStageRecs] staged candidates (0 = empty slot)
-  uint64_t* s_win = s_dyn + kStageRecs;  // [kWinCap] winners in bucket order / sort exchange
-  __shared__ __align__(16) uint32_t s_hist[2048];
-  __shared__ __align__(16) uint32_t s_cur[2048];
+  uint64_t* s_rec = s_dyn;              // [kSelStage] staged records, then winners in bucket order
+  uint64_t* s_out = s_dyn + kSelStage;  // [kMaxTopk] the row's output in order / radix winners
+  __shared__ __align__(16) uint32_t s_hist[kSelBins];
+  __shared__ __align__(16) uint32_t s_cur[kSelBins];
+  __shared__ int s_segoff[kSelSegs + 1];
+  __shared__ const uint64_t* s_segptr[kSelSegs];
   __shared__ int s_scratch[NT / 32];
   __shared__ int s_res[4];
-  __shared__ int s_n, s_staged, s_pos, s_maxc;
-  __shared__ unsigned long long s_lo, s_hi;
-  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ int s_total, s_n, s_pos, s_maxc;
+  __shared__ unsigned long long s_thr, s_lo, s_hi;
 
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  if (p.row_flags && p.row_flags[row] == 0) return;  // row already exact
+  if (p.skip && *p.skip) return;
+  // with row flags, write either the flagged rows (recovery) or the others
+  if (p.row_flags && ((p.row_flags[row] != 0) == (p.skip_flagged != 0))) return;
   const RowUnits R = row_units(p, row);
   const int G = (p.mode == kModeDecode) ? 1 : p.G;
   const CandLayout lay = p.lay;
 
   // segment sg = 5 * unit + region of the row's candidate buffers; one more
   // segment holds the row's extra records when given
+  auto unit_meta = [&](int u) -> const int32_t* {
+    return p.meta + (static_cast<size_t>(R.slot_lo + u) * G + R.q) * kMetaInts;
+  };
   auto segment = [&](int sg, int& cnt) -> const uint64_t* {
     if (sg == 5 * R.n_u) {
       cnt = p.topk;
@@ -190,88 +208,116 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
            lay.region_off(r);
   };
   const int n_seg = 5 * R.n_u + (p.extra_rec ? 1 : 0);
+  const bool table = n_seg <= kSelSegs;
 
-  // warp 0 sizes the segments (one lane per segment, a warp scan for the
-  // staging offsets) and, when they fit, issues one bulk copy per segment
-  // into consecutive 16-byte aligned slots
+  // 1. warp 0: segment table (offsets of a flattened index), total count and
+  //    the row threshold (largest unit threshold; the extra segment, sorted,
+  //    holds k records >= its k-th)
   if (wid == 0) {
-    int n = 0, staged = 0;
+    uint64_t thr = 0;
+    int off = 0;
     for (int base = 0; base < n_seg; base += 32) {
+      const int sg = base + lane;
       int c = 0;
-      if (base + lane < n_seg) segment(base + lane, c);
-      int c2 = (c + 1) & ~1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-        c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
+      const uint64_t* ptr = nullptr;
+      if (sg < n_seg) {
+        ptr = segment(sg, c);
+        if (sg == 5 * R.n_u) {
+          const uint64_t kth = ptr[p.topk - 1];
+          thr = kth > thr ? kth : thr;
+        } else if (sg % 5 == 0) {
+          const int32_t* mt = unit_meta(sg / 5);
+          const uint64_t ut = (static_cast<uint64_t>(static_cast<uint32_t>(mt[7])) << 32) |
+                              static_cast<uint64_t>(static_cast<uint32_t>(mt[6]));
+          thr = ut > thr ? ut : thr;
+        }
       }
-      n += c;
-      staged += c2;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (sg < n_seg && table) {
+        s_segoff[sg] = off + incl - c;
+        s_segptr[sg] = ptr;
+      }
+      off += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t v = __shfl_xor_sync(0xFFFFFFFFu, thr, o);
+      thr = v > thr ? v : thr;
     }
     if (lane == 0) {
-      s_n = n;
-      s_staged = staged;
+      s_total = off;
+      if (table) s_segoff[n_seg] = off;
+      s_thr = thr;
+      s_n = 0;
       s_pos = 0;
       s_maxc = 0;
       s_lo = ~0ull;
       s_hi = 0ull;
     }
-    if (staged <= kStageRecs && n > 0) {
-      const uint32_t bar = smem_u32(&s_bar);
-      if (lane == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(staged) * 8u);
+  }
+  __syncthreads();
+  const int total = s_total;
+  const uint64_t thr = s_thr;
+
+  // 2. one coalesced pass: count and stage the records at or above the row
+  //    threshold, tracking their score-code range
+  {
+    uint32_t clo = 0xFFFFFFFFu, chi = 0u;
+    auto take = [&](bool in, uint64_t r) {
+      const bool keep = in && r != 0ull && r >= thr;
+      stage_append(keep, r, s_rec, kSelStage, &s_n, lane);
+      if (keep) {
+        const uint32_t c = static_cast<uint32_t>(r >> 32);
+        clo = min(clo, c);
+        chi = max(chi, c);
       }
-      __syncwarp();
-      int off = 0;
-      for (int base = 0; base < n_seg; base += 32) {
-        int c = 0;
-        const uint64_t* src = nullptr;
-        if (base + lane < n_seg) src = segment(base + lane, c);
-        const int c2 = (c + 1) & ~1;
-        int incl = c2;
+    };
+    if (table) {
+      const int nsg = n_seg;
+      for (int base = 0; base < total; base += kBatch * NT) {
+        uint64_t r[kBatch];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
+        for (int j = 0; j < kBatch; ++j) {
+          const int i = base + j * NT + tid;
+          r[j] = 0ull;
+          if (i < total) {
+            int lo = 0, hi = nsg - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (s_segoff[mid] <= i) lo = mid; else hi = mid - 1;
+            }
+            r[j] = s_segptr[lo][i - s_segoff[lo]];
+          }
         }
-        if (c2 > 0) bulk_load(smem_u32(s_rec + off + incl - c2), src, static_cast<uint32_t>(c2) * 8u, bar);
-        off += __shfl_sync(0xFFFFFFFFu, incl, 31);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) take(base + j * NT + tid < total, r[j]);
       }
+    } else {
+      for (int sg = 0; sg < n_seg; ++sg) {
+        int cnt;
+        const uint64_t* buf = segment(sg, cnt);
+        for (int base = 0; base < cnt; base += NT) {
+          const int i = base + tid;
+          take(i < cnt, i < cnt ? buf[i] : 0ull);
+        }
+      }
+    }
+    clo = __reduce_min_sync(0xFFFFFFFFu, clo);
+    chi = __reduce_max_sync(0xFFFFFFFFu, chi);
+    if (lane == 0 && chi != 0u) {
+      atomicMin(&s_lo, static_cast<unsigned long long>(clo) << 32);
+      atomicMax(&s_hi, (static_cast<unsigned long long>(chi) << 32) | 0xFFFFFFFFull);
     }
   }
   __syncthreads();
-  const int n = s_n;
+  const int n = s_n;  // records at or above the row threshold
   const int m = min(p.topk, n);
-  const bool staged = s_staged <= kStageRecs;
-  const int n_st = staged ? s_staged : 0;
-
-  if (staged && n > 0) {
-    // warp 0 alone waits for the copies (the other warps park at the barrier
-    // below instead of spinning on the mbarrier) and blanks the padding slot
-    // after each odd-sized segment
-    if (wid == 0) {
-      volatile int never = 0;
-      mbar_wait(smem_u32(&s_bar), 0, &never, p.err);
-      __syncwarp();
-      int off = 0;
-      for (int base = 0; base < n_seg; base += 32) {
-        int c = 0;
-        if (base + lane < n_seg) segment(base + lane, c);
-        const int c2 = (c + 1) & ~1;
-        int incl = c2;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        if (c & 1) s_rec[off + incl - 1] = 0ull;
-        off += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-    }
-    __syncthreads();
-  }
+  const bool staged = n <= kSelStage;
 
   const size_t o = static_cast<size_t>(row) * p.topk;
   const size_t orec = static_cast<size_t>(row) * p.rec_stride;
@@ -284,49 +330,23 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   };
   if (p.out_kth && m == 0 && tid == 0) p.out_kth[row] = -INFINITY;
 
-  // ---- counting path
+  // 3. counting path over the staged records
   bool done = false;
   if (staged && m > 0) {
-    // every pass over the staged records takes kBatch of them per thread at a
-    // time, loads first, so that their shared-memory latencies overlap.
-    // First the row's smallest and largest score code (the high words;
-    // padding slots are 0 and wrap to the top under c - 1)
-    const uint32_t* s_code = reinterpret_cast<const uint32_t*>(s_rec);
-    uint32_t clo = 0xFFFFFFFFu, chi = 0u;
-    for (int base = tid; base < n_st; base += kBatch * NT) {
-      uint32_t c[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) c[j] = base + j * NT < n_st ? s_code[2 * (base + j * NT) + 1] : 0u;
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        clo = min(clo, c[j] - 1u);
-        chi = max(chi, c[j]);
-      }
-    }
-    clo = __reduce_min_sync(0xFFFFFFFFu, clo);
-    chi = __reduce_max_sync(0xFFFFFFFFu, chi);
-    for (int i = tid; i < 2048; i += NT) s_hist[i] = 0u;
-    if (lane == 0) {
-      atomicMin(&s_lo, static_cast<unsigned long long>(clo + 1u) << 32);
-      atomicMax(&s_hi, (static_cast<unsigned long long>(chi) << 32) | 0xFFFFFFFFull);
-    }
-    __syncthreads();
-    // bucket of a record: linear in its score between the row's smallest and
-    // largest score (any digit that never decreases along the record order
-    // works; a linear one spreads the winners evenly), or, when that range is
-    // zero or not finite, the top 11 bits of (record - smallest record)
+    for (int i = tid; i < kSelBins; i += NT) s_hist[i] = 0u;
+    // bucket of a record: linear in its score between the staged minimum and
+    // maximum (any digit that never decreases along the record order keeps
+    // the selection exact; a linear one spreads the winners evenly), or, when
+    // that range is zero or not finite, the top 10 bits of (record - smallest)
     const float smin = record_score(s_lo), srange = record_score(s_hi) - smin;
-    const float scale = 2047.0f / srange;
+    const float scale = static_cast<float>(kSelBins - 1) / srange;
     const bool lin = srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f;
     if (!lin) {
-      // equal (or non-finite) extreme scores: the exact record range instead
       uint64_t lo = ~0ull, hi = 0ull;
-      for (int i = tid; i < n_st; i += NT) {
+      for (int i = tid; i < n; i += NT) {
         const uint64_t r = s_rec[i];
-        if (r != 0ull) {
-          lo = r < lo ? r : lo;
-          hi = r > hi ? r : hi;
-        }
+        lo = r < lo ? r : lo;
+        hi = r > hi ? r : hi;
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -344,31 +364,28 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
         atomicMin(&s_lo, static_cast<unsigned long long>(lo));
         atomicMax(&s_hi, static_cast<unsigned long long>(hi));
       }
-      __syncthreads();
     }
+    __syncthreads();
     const uint64_t rlo = s_lo;
     const uint64_t span = s_hi - rlo;
-    const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 11);  // span >> shift < 2048
+    const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 10);  // span >> shift < 1024
     auto digit = [&](uint64_t r) {
-      if (lin) return min(2047u, static_cast<uint32_t>((record_score(r) - smin) * scale));
+      if (lin) return min(static_cast<uint32_t>(kSelBins - 1), static_cast<uint32_t>((record_score(r) - smin) * scale));
       return static_cast<uint32_t>((r - rlo) >> shift);
     };
-    for (int base = tid; base < n_st; base += kBatch * NT) {
+    for (int base = tid; base < n; base += kBatch * NT) {
       uint64_t r[kBatch];
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
+      for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n ? s_rec[base + j * NT] : 0ull;
 #pragma unroll
       for (int j = 0; j < kBatch; ++j)
         if (r[j] != 0ull) atomicAdd(&s_hist[digit(r[j])], 1u);
     }
     __syncthreads();
-    // descending exclusive scan: thread t owns buckets 2047-8t down to 2040-8t
-    const uint4 ha = reinterpret_cast<const uint4*>(s_hist)[(2040 - 8 * tid) >> 2];
-    const uint4 hb = reinterpret_cast<const uint4*>(s_hist)[(2044 - 8 * tid) >> 2];
-    const uint32_t c[8] = {hb.w, hb.z, hb.y, hb.x, ha.w, ha.z, ha.y, ha.x};
-    uint32_t sum = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sum += c[j];
+    // descending exclusive scan: thread t owns buckets 1023-4t down to 1020-4t
+    const uint4 h4 = reinterpret_cast<const uint4*>(s_hist)[(kSelBins - 4 - 4 * tid) >> 2];
+    const uint32_t c[4] = {h4.w, h4.z, h4.y, h4.x};
+    const uint32_t sum = c[0] + c[1] + c[2] + c[3];
     uint32_t incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -379,11 +396,11 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     __syncthreads();
     uint32_t run = incl - sum;
     for (int w2 = 0; w2 < wid; ++w2) run += static_cast<uint32_t>(s_scratch[w2]);
-    uint32_t ex[8];
+    uint32_t ex[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
       ex[j] = run;
-      const int d = 2047 - 8 * tid - j;
+      const int d = kSelBins - 1 - 4 * tid - j;
       if (c[j] > 0u && run <= static_cast<uint32_t>(m - 1) && static_cast<uint32_t>(m - 1) < run + c[j]) {
         s_res[0] = d;
         s_res[1] = static_cast<int>(run);
@@ -391,45 +408,42 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       }
       run += c[j];
     }
-    reinterpret_cast<uint4*>(s_cur)[(2040 - 8 * tid) >> 2] = make_uint4(ex[7], ex[6], ex[5], ex[4]);
-    reinterpret_cast<uint4*>(s_cur)[(2044 - 8 * tid) >> 2] = make_uint4(ex[3], ex[2], ex[1], ex[0]);
+    reinterpret_cast<uint4*>(s_cur)[(kSelBins - 4 - 4 * tid) >> 2] = make_uint4(ex[3], ex[2], ex[1], ex[0]);
     __syncthreads();
     const int B = s_res[0], above = s_res[1], cntB = s_res[2];
     uint32_t mc = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (2047 - 8 * tid - j >= B) mc = c[j] > mc ? c[j] : mc;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint32_t v = __shfl_xor_sync(0xFFFFFFFFu, mc, off);
-      mc = v > mc ? v : mc;
-    }
+    for (int j = 0; j < 4; ++j)
+      if (kSelBins - 1 - 4 * tid - j >= B) mc = c[j] > mc ? c[j] : mc;
+    mc = __reduce_max_sync(0xFFFFFFFFu, mc);
     if (lane == 0) atomicMax(&s_maxc, static_cast<int>(mc));
     __syncthreads();
     const int nw = above + cntB;  // records in bucket B and above
-    if (nw <= kWinCap && s_maxc <= kRankMax) {
-      for (int base = tid; base < n_st; base += kBatch * NT) {
-        uint64_t r[kBatch];
-        uint32_t pos[kBatch];
+    if (s_maxc <= kRankMax) {
+      // scatter the winners into bucket order, in place: every thread holds
+      // its records in registers across the barrier
+      constexpr int kPer = kSelStage / NT;
+      uint64_t v[kPer];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < n_st ? s_rec[base + j * NT] : 0ull;
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-          const uint32_t d = r[j] != 0ull ? digit(r[j]) : 0u;
-          pos[j] = (r[j] != 0ull && static_cast<int>(d) >= B) ? atomicAdd(&s_cur[d], 1u) : 0xFFFFFFFFu;
-        }
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j)
-          if (pos[j] != 0xFFFFFFFFu) s_win[pos[j]] = r[j];
+      for (int j = 0; j < kPer; ++j) {
+        const int i = j * NT + tid;
+        v[j] = i < n ? s_rec[i] : 0ull;
       }
       __syncthreads();
-      // s_cur[d] is now the end of bucket d; rank each record inside its
-      // bucket and place the winners in order in the (now free) staging buffer
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if (v[j] == 0ull) continue;
+        const uint32_t d = digit(v[j]);
+        if (static_cast<int>(d) >= B) s_rec[atomicAdd(&s_cur[d], 1u)] = v[j];
+      }
+      __syncthreads();
+      // s_cur[d] is now the end of bucket d; rank each winner inside its
+      // bucket and place it at its final position of the output
       for (int base = tid; base < nw; base += kBatch * NT) {
         uint64_t r[kBatch];
         int beg[kBatch], end[kBatch];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < nw ? s_win[base + j * NT] : 0ull;
+        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < nw ? s_rec[base + j * NT] : 0ull;
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
           const uint32_t d = r[j] != 0ull ? digit(r[j]) : 0u;
@@ -446,37 +460,32 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
         for (int x = 0; x < len; x += 2) {
 #pragma unroll
           for (int j = 0; j < kBatch; ++j) {
-            const uint64_t a0 = beg[j] + x < end[j] ? s_win[beg[j] + x] : 0ull;
-            const uint64_t a1 = beg[j] + x + 1 < end[j] ? s_win[beg[j] + x + 1] : 0ull;
+            const uint64_t a0 = beg[j] + x < end[j] ? s_rec[beg[j] + x] : 0ull;
+            const uint64_t a1 = beg[j] + x + 1 < end[j] ? s_rec[beg[j] + x + 1] : 0ull;
             rank[j] += (a0 > r[j] ? 1 : 0) + (a1 > r[j] ? 1 : 0);
           }
         }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j)
-          if (r[j] != 0ull && beg[j] + rank[j] < m) s_rec[beg[j] + rank[j]] = r[j];
+          if (r[j] != 0ull && beg[j] + rank[j] < m) s_out[beg[j] + rank[j]] = r[j];
       }
       __syncthreads();
-      for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_rec[i] : 0ull);
+      for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_out[i] : 0ull);
       done = true;
     }
     __syncthreads();
   }
   if (done) return;
 
-  // ---- radix-select + bitonic-sort path
-  uint64_t thr = 1;  // records are >= 1: keeps all
+  // 4. radix-select + bitonic-sort path (rows with more records than the
+  //    staging buffer, or with crowded buckets): over the staged records or
+  //    the buffers themselves, records below the row threshold skipped
+  uint64_t rthr = thr > 1ull ? thr : 1ull;  // records are >= 1
   if (m > 0 && m < n) {
     uint64_t prefix = 0;
     int pbits = 0, above = 0;
-    if (staged) {
-      // start the digits at the highest bit in which the records differ
-      // (s_lo / s_hi bracket the records; the counting path reduced them)
-      const uint64_t diff = s_lo ^ s_hi;  // non-zero: records are distinct
-      pbits = __clzll(static_cast<long long>(diff));
-      prefix = pbits > 0 ? (s_hi >> (64 - pbits)) : 0ull;
-    }
-    for (int pass = 0; pass < 7; ++pass) {
-      const int shift = max(64 - pbits - 11, 0);
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = max(64 - pbits - 10, 0);
       const int width = 64 - pbits - shift;
       const int nb = 1 << width;
       for (int i = tid; i < nb; i += NT) s_hist[i] = 0;
@@ -491,14 +500,14 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            bool ok = v[j] != 0ull;
+            bool ok = v[j] != 0ull && v[j] >= thr;
             if (pbits > 0) ok = ok && ((v[j] >> (64 - pbits)) == prefix);
-            hist_add_blk(s_hist, ok, static_cast<uint32_t>(v[j] >> shift) & static_cast<uint32_t>(nb - 1));
+            if (ok) atomicAdd(&s_hist[static_cast<uint32_t>(v[j] >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
           }
         }
       };
       if (staged) {
-        hist_pass(s_rec, n_st);
+        hist_pass(s_rec, n);
       } else {
         for (int sg = 0; sg < n_seg; ++sg) {
           int cnt;
@@ -512,7 +521,7 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
       prefix = (prefix << width) | static_cast<uint64_t>(B);
       pbits += width;
       if (new_above + cnt == m || pbits == 64) {
-        thr = (pbits == 64) ? prefix : (prefix << (64 - pbits));
+        rthr = (pbits == 64) ? prefix : (prefix << (64 - pbits));
         break;
       }
       above = new_above;
@@ -520,24 +529,24 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
     }
   }
 
-  // gather the m winners (in any order) into s_win
+  // gather the m winners (in any order) into s_out
   auto gather = [&](const uint64_t* buf, int cnt) {
     for (int base = 0; base < cnt; base += NT) {
       const int i = base + tid;
       const uint64_t r = (i < cnt) ? buf[i] : 0ull;
-      const bool keep = (i < cnt) && (r >= thr) && (r != 0ull);
+      const bool keep = (i < cnt) && (r >= rthr) && (r >= thr) && (r != 0ull);
       const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
       if (bal) {
         int pos = 0;
         if (lane == 0) pos = atomicAdd(&s_pos, __popc(bal));
         pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
         const int at = pos + __popc(bal & lanemask_lt());
-        if (keep && at < kMaxTopk) s_win[at] = r;
+        if (keep && at < kMaxTopk) s_out[at] = r;
       }
     }
   };
   if (staged) {
-    gather(s_rec, n_st);
+    gather(s_rec, n);
   } else {
     for (int sg = 0; sg < n_seg; ++sg) {
       int cnt;
@@ -549,33 +558,32 @@ __global__ void __launch_bounds__(NT) select_topk_kernel(const SelectParams p) {
   if (tid == 0 && s_pos != m) atomicOr(p.err, kErrOverflow);  // never expected
   uint64_t v[8];
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int i = 8 * tid + s;
-    v[s] = (i < m) ? s_win[i] : 0ull;
+  for (int s2 = 0; s2 < 8; ++s2) {
+    const int i = 8 * tid + s2;
+    v[s2] = (i < m) ? s_out[i] : 0ull;
   }
   __syncthreads();
-  sort2048_desc(v, s_win);
+  sort2048_desc(v, s_rec);
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int i = 8 * tid + s;
-    if (i < p.topk) put(i, i < m ? v[s] : 0ull);
+  for (int s2 = 0; s2 < 8; ++s2) {
+    const int i = 8 * tid + s2;
+    if (i < p.topk) put(i, i < m ? v[s2] : 0ull);
   }
 }
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   if (p.n_rows <= 0) return cudaSuccess;
   constexpr int NT = kSelectThreads;
-  const size_t smem = (kStageRecs + kWinCap) * sizeof(uint64_t);
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
+  if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(select_topk_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+                                         static_cast<int>(kSelectSmem));
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    if (dev >= 0 && dev < 64) configured[dev].store(true, std::memory_order_release);
   }
-  select_topk_kernel<NT><<<static_cast<unsigned>(p.n_rows), NT, smem, stream>>>(p);
+  select_topk_kernel<NT><<<static_cast<unsigned>(p.n_rows), NT, kSelectSmem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -211,6 +211,26 @@ def test_device_status_clean_after_calls():
     assert dsa.dsa_index_device_status(ws) == 0
 
 
+def test_prefill_row_blocks_match_one_launch():
+    # a workspace smaller than the chunk needs: the call runs consecutive
+    # launches over row blocks; rows are independent, so the output equals
+    # the single-launch output bit for bit
+    T_q, off, topk = 3000, 1000, 256
+    x = make_prefill("causal_16k_h64", T_q=T_q, T_k=off + T_q, q_offset=off, seed=71)
+    q, w, k = bf16(x["q"]), f32(x["w"]), bf16(x["k"])
+    full_idx, full_sc = dsa.dsa_index_prefill(q, w, k, off, topk)
+    small = dsa.dsa_index_prefill_workspace_bytes(700, off + T_q, 64, 128, topk)
+    assert small < dsa.dsa_index_prefill_workspace_bytes(T_q, off + T_q, 64, 128, topk)
+    ws = torch.empty(small, dtype=torch.uint8, device="cuda")
+    idx, sc = dsa.dsa_index_prefill(q, w, k, off, topk, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, full_idx) and torch.equal(sc.view(torch.int32), full_sc.view(torch.int32))
+    assert dsa.dsa_index_device_status(ws) == 0
+    # a workspace below one query group is refused
+    with pytest.raises(dsa.DSAError, match="EWORKSPACE"):
+        dsa.dsa_index_prefill(q, w, k, off, topk, workspace=torch.empty(1 << 16, dtype=torch.uint8, device="cuda"))
+
+
 # ---------------------------------------------------------------- full sizes
 
 def _sample_rows(T_q, n):
@@ -239,3 +259,18 @@ def test_full_size_decode_sampled_sequences():
     oi, osc, amax, score_of = oracle_decode_rows(sub, wl.topk)
     check_rows(idx.cpu().numpy()[pick], sc.cpu().numpy()[pick], oi, osc, amax, sub["seq_len"],
                wl.topk, score_of, "decode full")
+
+
+def test_full_size_32k_row_chunk_against_1m_keys_in_row_blocks():
+    # a 32K-row chunk at the end of a 1M context with a 512 MiB workspace:
+    # the call runs in row blocks; sampled rows match the oracle
+    T_q, T_k = 32768, 1 << 20
+    x = make_prefill("chunk_1m_h64", T_q=T_q, T_k=T_k, q_offset=T_k - T_q, seed=72)
+    ws = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    idx, sc = dsa.dsa_index_prefill(bf16(x["q"]), f32(x["w"]), bf16(x["k"]), x["q_offset"], 2048, workspace=ws)
+    torch.cuda.synchronize()
+    assert dsa.dsa_index_device_status(ws) == 0
+    rows = _sample_rows(T_q, 5)
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, 2048)
+    check_rows(idx.cpu().numpy()[rows], sc.cpu().numpy()[rows], oi, osc, amax, x["q_offset"] + rows + 1, 2048,
+               score_of, "32K rows x 1M keys")

@@ -37,13 +37,31 @@ def anchor_seeds(x, topk, n_random, seed):
     return np.concatenate([anchor, rnd]).astype(np.int32)
 
 
-def run_both(x, topk, seeds):
+PROBE_ROWS = 64  # rows of a chunk longer than 128 rows that always take the pruned path
+
+
+def run_both(x, topk, seeds, workspace=None):
     q, w, k = dev_inputs(x)
     di, ds = dsa.dsa_index_prefill(q, w, k, x["q_offset"], topk)
     pi, ps, st = dsa.dsa_index_prefill_pruned(q, w, k, x["q_offset"], topk,
-                                              torch.from_numpy(seeds).cuda(), stats=True)
+                                              torch.from_numpy(seeds).cuda(), stats=True,
+                                              workspace=workspace)
     torch.cuda.synchronize()
     return di.cpu().numpy(), ds.cpu().numpy(), pi.cpu().numpy(), ps.cpu().numpy(), st
+
+
+def screened_rows(T_q, st):
+    """Rows that went through the screen: all of them, or only the probe when
+    the probe sent the rest of the chunk to the dense pass."""
+    if st["bypassed_rows"] == 0:
+        return T_q
+    assert T_q > 2 * PROBE_ROWS and st["bypassed_rows"] == T_q - PROBE_ROWS
+    return PROBE_ROWS
+
+
+def expected_screened_pairs(off, T_q, n_seed, st):
+    n = screened_rows(T_q, st)
+    return sum(off + t + 1 - n_seed for t in range(n))
 
 
 @pytest.mark.parametrize("recipe,H", [("causal_1k_h64", 64), ("causal_16k_h64", 64),
@@ -59,8 +77,7 @@ def test_pruned_equals_dense_bitwise_and_oracle(recipe, H):
     oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
     check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, f"pruned {recipe}")
     T_q = T_k - off
-    vis = (2 * off + T_q + 1) * T_q // 2
-    assert st["screened_pairs"] == vis - T_q * len(seeds)
+    assert st["screened_pairs"] == expected_screened_pairs(off, T_q, len(seeds), st)
     assert 0 <= st["survivor_pairs"] <= st["screened_pairs"]
     assert st["refined_pairs"] <= st["survivor_pairs"]
     print(recipe, st)
@@ -124,7 +141,7 @@ def test_pruned_ragged_chunk_and_small_topk():
 
 def test_pruned_overflowing_rows_are_recovered_exactly():
     # only topk random seeds: tau is weak, survivors exceed the per-row list
-    # (max(T_k/4, 4 topk) = 2048 keys), and those rows take the dense path
+    # (max(T_k/16, 4 topk) = 514 keys), and those rows take the dense path
     x = make_prefill("causal_1k_h64", T_q=40, T_k=8232, q_offset=8192, seed=9)
     seeds = random_distinct_keys(3, 0, 8192, 64)
     di, ds, pi, ps, st = run_both(x, 64, seeds)
@@ -162,3 +179,134 @@ def test_full_size_pruned_equals_dense(name, n_rows):
     oi, osc, amax, score_of = oracle_prefill_rows(x, rows, wl.topk)
     check_rows(pi[rows], ps[rows], oi, osc, amax, wl.q_offset + rows + 1, wl.topk, score_of, name)
     print(name, st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
+
+
+def _oracle_row_scores(x, row, n_keys):
+    return oracle.row_scores(x["q"][row], x["w"][row], x["k"], n_keys)
+
+
+def check_screen_safety(x, topk, seeds, ws, st, rows):
+    """Every key the GPU screen pruned scores (exactly, in fp64) strictly below
+    the row's GPU threshold tau ("DoSA", step 2: prune only when the bound is
+    below the threshold; the bound never underestimates a score), and tau is
+    the row's topk-th seed score up to the parity tolerance."""
+    off, T_q, T_k, H = x["q_offset"], x["q"].shape[0], x["k"].shape[0], x["H"]
+    mask, tau, state = dsa.dsa_index_prefill_pruned_survivors(ws, T_q, T_k, off, H, 128, topk, len(seeds))
+    torch.cuda.synchronize()
+    mask = mask.cpu().numpy().view(np.uint32)
+    tau, state = tau.cpu().numpy(), state.cpu().numpy()
+    is_seed = np.zeros(T_k, bool)
+    is_seed[seeds] = True
+    checked = 0
+    for t in rows:
+        assert state[t] in (0, 1), f"row {t} was not screened (state {state[t]})"
+        nvis = off + t + 1
+        bits = ((mask[t][np.arange(nvis) >> 5] >> (np.arange(nvis) & 31)) & 1).astype(bool)
+        assert not (bits & is_seed[:nvis]).any(), "seed keys must not appear as screened survivors"
+        I = _oracle_row_scores(x, t, nvis)
+        pruned = ~bits & ~is_seed[:nvis]
+        worst = float(I[pruned].max()) if pruned.any() else -np.inf
+        assert worst < float(tau[t]), f"row {t}: pruned key scores {worst} >= tau {tau[t]}"
+        seed_sc = np.sort(I[seeds])[::-1]
+        tol = 2e-3 * float(np.abs(I).max())
+        assert abs(float(tau[t]) - seed_sc[topk - 1]) <= tol, (t, tau[t], seed_sc[topk - 1])
+        checked += int(pruned.sum())
+    return checked
+
+
+@pytest.mark.parametrize("recipe,head_rank", [("causal_1k_h64", 0), ("causal_16k_h64", 1)])
+def test_screen_prunes_only_keys_below_tau_tiny_chunk(recipe, head_rank):
+    # 1024 keys split at q_offset = 512 (the oracle-sized shape; the shared
+    # latent heads let the bound prune): every screened row, every visible
+    # key checked against the fp64 scores
+    off, T_k, topk = 512, 1024, 256
+    x = make_prefill(recipe, T_q=T_k - off, T_k=T_k, q_offset=off, seed=21, head_rank=head_rank)
+    seeds = random_distinct_keys(22, 0, off, 384)
+    ws = torch.zeros(dsa.dsa_index_prefill_pruned_workspace_bytes(T_k - off, T_k, 64, 128, topk, len(seeds)),
+                     dtype=torch.uint8, device="cuda")
+    di, ds, pi, ps, st = run_both(x, topk, seeds, workspace=ws)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    n = screened_rows(T_k - off, st)
+    pruned = check_screen_safety(x, topk, seeds, ws, st, range(n))
+    print("tiny chunk", recipe, head_rank, "pruned keys checked", pruned, st)
+    if head_rank:
+        assert pruned > 0
+
+
+@pytest.mark.parametrize("head_rank", [0, 1])
+def test_screen_prunes_only_keys_below_tau_full_size_128k(head_rank):
+    # the 128K / H32 chunk at full size (8192 rows x 131072 keys, the
+    # benchmark's seed recipe); rows spread over the screened ones
+    wl = WORKLOADS["chunk_128k_h32"]
+    x = make_prefill(wl, with_anchor=True, head_rank=head_rank)
+    seeds = anchor_seeds(x, wl.topk, wl.n_seed - wl.n_anchor, seed=11)
+    ws = torch.zeros(dsa.dsa_index_prefill_pruned_workspace_bytes(wl.T_q, wl.T_k, wl.H, 128, wl.topk, wl.n_seed),
+                     dtype=torch.uint8, device="cuda")
+    di, ds, pi, ps, st = run_both(x, wl.topk, seeds, workspace=ws)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    n = screened_rows(wl.T_q, st)
+    rows = np.unique(np.linspace(0, n - 1, 6).round().astype(np.int64))
+    pruned = check_screen_safety(x, wl.topk, seeds, ws, st, rows)
+    print("128K chunk head_rank", head_rank, "pruned keys checked", pruned, st)
+
+
+def _tight_bound_chunk(wl_name, T_q, T_k, off, topk, seed, n_random):
+    """Rows repeating one query built so that the DoSA bound is exact up to its
+    safety slack: 14 distinct heads with large weights (the planner retains
+    them) and H-14 identical copies of one vector with small negative weights
+    (no positive omitted head; folding identical negative heads loses
+    nothing).  The seeds hold the query's Top-k among the keys before the
+    chunk, so tau is close to every row's k-th score."""
+    x = make_prefill(wl_name, T_q=T_q, T_k=T_k, q_offset=off, seed=seed)
+    H = x["H"]
+    rng = np.random.default_rng(0)
+    q0 = x["q"][0].copy()
+    q0[14:] = q0[14]
+    w0 = np.empty(H, np.float32)
+    w0[:14] = rng.standard_normal(14).astype(np.float32) * 4.0
+    w0[14:] = -0.01
+    x["q"][:] = q0
+    x["w"][:] = w0
+    idx, _, _ = oracle.prefill_topk(x["q"][:1], x["w"][:1], x["k"][:off], off - 1, topk)
+    seeds = np.concatenate([idx[0], random_distinct_keys(13, 0, off, n_random, exclude=idx[0])]).astype(np.int32)
+    return x, seeds
+
+
+def test_full_size_pruned_refine_path_without_recovery():
+    # the 128K / H32 chunk's sizes (8192 rows x 131072 keys, 12288 seeds) with
+    # the constructed tight-bound heads: the probe keeps the pruned path, no
+    # row overflows, the result comes from screen -> compact -> refine and is
+    # bit for bit the dense one
+    wl = WORKLOADS["chunk_128k_h32"]
+    x, seeds = _tight_bound_chunk("chunk_128k_h32", wl.T_q, wl.T_k, wl.q_offset, wl.topk, 408,
+                                  wl.n_seed - wl.topk)
+    assert len(seeds) == wl.n_seed
+    ws = torch.zeros(dsa.dsa_index_prefill_pruned_workspace_bytes(wl.T_q, wl.T_k, wl.H, 128, wl.topk, wl.n_seed),
+                     dtype=torch.uint8, device="cuda")
+    di, ds, pi, ps, st = run_both(x, wl.topk, seeds, workspace=ws)
+    print("full-size tight bound", st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    assert st["bypassed_rows"] == 0 and st["recovered_rows"] == 0
+    assert st["refined_pairs"] == st["survivor_pairs"] > 0
+    assert st["screened_pairs"] == expected_screened_pairs(wl.q_offset, wl.T_q, wl.n_seed, st)
+    rows = np.array([0, 4095, wl.T_q - 1])
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, wl.topk)
+    check_rows(pi[rows], ps[rows], oi, osc, amax, wl.q_offset + rows + 1, wl.topk, score_of, "tight full")
+    check_screen_safety(x, wl.topk, seeds, ws, st, rows)
+
+
+def test_probe_sends_an_unfilterable_chunk_to_the_dense_pass():
+    # the 128K recipe (independent heads: the bound filters little) on a 1024
+    # row chunk: the 128 probe rows are screened, the rest skip the pruned
+    # path; the result is still the dense one bit for bit
+    off, T_q, topk = 15360, 1024, 512
+    x = make_prefill("chunk_128k_h32", T_q=T_q, T_k=off + T_q, q_offset=off, seed=33, with_anchor=True)
+    seeds = anchor_seeds(x, topk, 2560, seed=34)
+    di, ds, pi, ps, st = run_both(x, topk, seeds)
+    print("bypass", st)
+    assert st["bypassed_rows"] == T_q - PROBE_ROWS
+    assert st["screened_pairs"] == expected_screened_pairs(off, T_q, len(seeds), st)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    rows = np.array([0, 127, 128, 700, T_q - 1])
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
+    check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, "bypass")

@@ -329,8 +329,59 @@ def test_dosa_row_is_lossless_and_the_bound_is_safe(recipe, r, sign):
 
 
 def test_planner_sample_positions():
+    # "DoSA" reading notes, annotation ADQKPC5Q, step 1: the planner samples
+    # 128 positions 32 + 64 i of the seed region (12,288 seeds)
     seeds = np.arange(12288, dtype=np.int32) * 3
     s = oracle.dosa_sample(seeds)
-    assert s.shape == (128,)
-    assert s[0] == 3 * 48 and s[-1] == 3 * (48 + 96 * 127)
+    assert s.tolist() == [3 * (32 + 64 * i) for i in range(128)]
+    # shorter lists keep the even spacing: every entry when there are at most 128
     assert oracle.dosa_sample(seeds[:5]).tolist() == [0, 3, 6, 9, 12]
+    assert oracle.dosa_sample(seeds[:1024]).tolist() == [3 * (4 + 8 * i) for i in range(128)]
+
+
+# ------------------------------------------------------- pair scorer ------
+
+def test_score_pairs_matches_a_numpy_matmul_at_random_pairs():
+    # the per-pair scorer every GPU parity test uses: I(t, s) from the widened
+    # bf16/fp32 inputs by numpy (einsum + ReLU + weighted sum), at random
+    # (row, key) pairs, for a chunk layout (rows index q/w, keys index k) and
+    # for one decode sequence's cache
+    rng = np.random.default_rng(17)
+    for H, d in ((64, 128), (32, 128), (3, 8)):
+        T_q, T_k = 9, 300
+        q = bf16_bits_from_f64(rng.standard_normal((T_q, H, d)) / 4)
+        k = bf16_bits_from_f64(rng.standard_normal((T_k, d)))
+        w = rng.standard_normal((T_q, H)).astype(np.float32)
+        rows = rng.integers(0, T_q, size=200)
+        keys = rng.integers(0, T_k, size=200)
+        got = oracle.score_pairs(q, w, k, rows, keys)
+        Q = bf16_bits_to_f32(q).astype(np.float64)
+        K = bf16_bits_to_f32(k).astype(np.float64)
+        dots = np.einsum("nhd,nd->nh", Q[rows], K[keys])
+        ref = (w[rows].astype(np.float64) * np.maximum(dots, 0.0)).sum(axis=1)
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    # a wrong row or key stride would pick another vector: distinct rows and
+    # keys give distinct scores here, and swapping the two index lists changes
+    # the result
+    assert not np.allclose(oracle.score_pairs(q, w, k, rows, keys),
+                           oracle.score_pairs(q, w, k, rows[::-1], keys))
+
+
+def test_score_pairs_agrees_with_the_chunk_and_decode_scores():
+    # the same pairs scored through the chunked prefill (q_offset > 0) and the
+    # batched decode layouts give identical values
+    x = make_prefill("chunk_128k_h32", T_q=6, T_k=500, q_offset=494)
+    _, _, _, full = oracle.prefill_topk(x["q"], x["w"], x["k"], 494, 4, want_scores=True)
+    rng = np.random.default_rng(3)
+    rows = rng.integers(0, 6, size=50)
+    keys = np.array([rng.integers(0, 494 + r + 1) for r in rows])
+    got = oracle.score_pairs(x["q"], x["w"], x["k"], rows, keys)
+    assert (got == full[rows, keys]).all()
+    # decode: sequence b's query against its own cache
+    L = np.array([500, 300], np.int32)
+    kc = np.stack([x["k"], x["k"][::-1].copy()])
+    q, w = x["q"][:2], x["w"][:2]
+    idx, sc, _ = oracle.decode_topk(q, w, kc, L, 5)
+    for b in range(2):
+        got = oracle.score_pairs(q[b:b + 1], w[b:b + 1], kc[b], np.zeros(5, np.int64), idx[b])
+        assert (got == sc[b]).all()

@@ -52,3 +52,20 @@ def test_noalloc_decode_rejects_batches_above_its_static_limit():
     sl = torch.from_numpy(x["seq_len"]).cuda()
     with pytest.raises(dsa.DSAError, match="static scratch limit"):
         dsa.dsa_index_decode_noalloc(q, w, k, sl, 8)
+
+
+def test_noalloc_decode_reports_device_checks_in_its_own_status_word():
+    # the static scratch carries the device status word: a length above the
+    # cache capacity is treated as 0 and sets bit 1, readable without a
+    # workspace; the next clean call clears it
+    lens = [40, 17]
+    x = make_decode("decode_64x128k_h64", B=2, t_cap=40, seq_len=lens, seed=33)
+    q, w, k = _bf16(x["q"]), torch.from_numpy(x["w"]).cuda(), _bf16(x["k"])
+    bad = torch.tensor([40, 41], dtype=torch.int32, device="cuda")  # 41 > t_cap
+    idx, _ = dsa.dsa_index_decode_noalloc(q, w, k, bad, 8)
+    torch.cuda.synchronize()
+    assert dsa.dsa_index_decode_noalloc_status() & 2
+    assert (idx[1] == -1).all().item()  # the bad sequence sees no keys
+    sl = torch.from_numpy(x["seq_len"]).cuda()
+    dsa.dsa_index_decode_noalloc(q, w, k, sl, 8)
+    assert dsa.dsa_index_decode_noalloc_status() == 0
