@@ -58,6 +58,12 @@ def _load():
         _lib.oracle_dosa_row.argtypes = [P, P, P, I64, P, I32, I32, I32, I32, I32, P, P, P, P,
                                          P, P]
         _lib.oracle_dosa_row.restype = I32
+        U8 = P
+        _lib.oracle_e4m3_decode.argtypes = [U8, I64, P]
+        _lib.oracle_prefill_topk_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, I64,
+                                                 P, P, P, I32]
+        _lib.oracle_prefill_topk_fp8.restype = I32
+        _lib.oracle_score_pairs_fp8.argtypes = [P, P, P, P, P, I32, I32, I64, P, P, P, I32]
         for f in ("oracle_n_dense",):
             getattr(_lib, f).argtypes = [D]
             getattr(_lib, f).restype = D
@@ -138,6 +144,46 @@ def decode_topk(q, w, k, seq_len, topk: int, n_threads: int | None = None):
     if rc != 0:
         raise ValueError("oracle_decode_topk: bad arguments")
     return idx, sc, amax
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of FP8 E4M3 codes (uint8), in fp64."""
+    codes = _c(codes, np.uint8).ravel()
+    out = np.empty(codes.shape[0], np.float64)
+    _load().oracle_e4m3_decode(_p(codes), codes.shape[0], _p(out))
+    return out
+
+
+def prefill_topk_fp8(q, q_scale, w, k, k_scale, q_offset: int, topk: int, rows=None,
+                     n_threads: int | None = None):
+    """prefill_topk on FP8 inputs: q (T_q,H,d) / k (T_k,d) E4M3 codes with fp32
+    scales q_scale (T_q,H) and k_scale (T_k,).  Returns (idx, score, absmax)."""
+    q, k = _c(q, np.uint8), _c(k, np.uint8)
+    q_scale, w, k_scale = _c(q_scale, np.float32), _c(w, np.float32), _c(k_scale, np.float32)
+    T_q, H, d = q.shape
+    T_k = k.shape[0]
+    rows = np.arange(T_q, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    n = rows.shape[0]
+    idx = np.empty((n, topk), np.int32)
+    sc = np.empty((n, topk), np.float64)
+    amax = np.empty(n, np.float64)
+    rc = _load().oracle_prefill_topk_fp8(_p(q), _p(q_scale), _p(w), _p(k), _p(k_scale), q_offset, T_q,
+                                         T_k, H, d, topk, _p(rows), n, _p(idx), _p(sc), _p(amax),
+                                         n_threads or threads())
+    if rc != 0:
+        raise ValueError("oracle_prefill_topk_fp8: bad arguments")
+    return idx, sc, amax
+
+
+def score_pairs_fp8(q, q_scale, w, k, k_scale, q_rows, keys, n_threads: int | None = None) -> np.ndarray:
+    q, k = _c(q, np.uint8), _c(k, np.uint8)
+    q_scale, w, k_scale = _c(q_scale, np.float32), _c(w, np.float32), _c(k_scale, np.float32)
+    q_rows, keys = _c(q_rows, np.int64).ravel(), _c(keys, np.int64).ravel()
+    H, d = q.shape[-2], q.shape[-1]
+    out = np.empty(q_rows.shape[0], np.float64)
+    _load().oracle_score_pairs_fp8(_p(q), _p(q_scale), _p(w), _p(k), _p(k_scale), H, d, q_rows.shape[0],
+                                   _p(q_rows), _p(keys), _p(out), n_threads or threads())
+    return out
 
 
 def dosa_sample(seeds) -> np.ndarray:

@@ -456,6 +456,87 @@ OR_API int oracle_dosa_row(const uint16_t *q_row, const float *w_row, const uint
   return 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * FP8 indexer scoring ("DeepSeek DSA FLOPs", Lightning Indexer: the indexer
+ * runs in FP8).  Reading: q and k are stored as FP8 E4M3 codes with one fp32
+ * scale per stored row (per query head row and per key), so the real vectors
+ * are q(t,j) = q_scale(t,j) * e4m3(q8(t,j)) and k(s) = k_scale(s) * e4m3(k8(s)),
+ * and the index score is the same definition on them:
+ *     I(t,s) = sum_j w(t,j) * ReLU(q(t,j) . k(s)).
+ * ------------------------------------------------------------------------ */
+/* OCP FP8 E4M3 ("FN"): sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ * exponent field 0 holds the subnormals m/8 * 2^-6; no infinities; the
+ * all-ones exponent and mantissa pattern is NaN. */
+static double e4m3_to_f64(uint8_t b) {
+  int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sgn ? -v : v;
+}
+
+OR_API void oracle_e4m3_decode(const uint8_t *codes, int64_t n, double *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_f64(codes[i]);
+}
+
+static double index_score_fp8(const uint8_t *q_row, const float *qs_row, const float *w_row,
+                              const uint8_t *k_s, double ks, int H, int d) {
+  double I = 0.0;
+  for (int j = 0; j < H; ++j) {
+    double x = 0.0, qs = (double)qs_row[j];
+    for (int i = 0; i < d; ++i)
+      x += (qs * e4m3_to_f64(q_row[(size_t)j * d + i])) * (ks * e4m3_to_f64(k_s[i]));
+    I += (double)w_row[j] * (x > 0.0 ? x : 0.0);
+  }
+  return I;
+}
+
+/* The FP8 chunked causal prefill: as oracle_prefill_topk, on FP8 inputs. */
+OR_API int oracle_prefill_topk_fp8(const uint8_t *q, const float *q_scale, const float *w,
+                                   const uint8_t *k, const float *k_scale, int64_t q_offset,
+                                   int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                   const int64_t *rows, int64_t n_rows, int32_t *out_idx,
+                                   double *out_score, double *out_absmax, int n_threads) {
+  if (q_offset < 0 || q_offset + T_q > T_k || topk <= 0) return -1;
+  for (int64_t i = 0; i < n_rows; ++i)
+    if (rows[i] < 0 || rows[i] >= T_q) return -1;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int64_t i = 0; i < n_rows; ++i) {
+    int64_t t = rows[i];
+    int64_t nvis = q_offset + t + 1;
+    rec_t *recs = (rec_t *)malloc(sizeof(rec_t) * (size_t)nvis);
+    double amax = 0.0;
+    for (int64_t s = 0; s < nvis; ++s) {
+      double I = index_score_fp8(q + (size_t)t * H * d, q_scale + (size_t)t * H, w + (size_t)t * H,
+                                 k + (size_t)s * d, (double)k_scale[s], H, d);
+      recs[s].score = I;
+      recs[s].key = s;
+      if (fabs(I) > amax) amax = fabs(I);
+    }
+    out_absmax[i] = amax;
+    emit_topk(recs, nvis, topk, out_idx + (size_t)i * topk, out_score + (size_t)i * topk);
+    free(recs);
+  }
+  return 0;
+}
+
+/* Scores of arbitrary (query row, key) pairs of FP8 inputs. */
+OR_API void oracle_score_pairs_fp8(const uint8_t *q, const float *q_scale, const float *w,
+                                   const uint8_t *k, const float *k_scale, int H, int d, int64_t n,
+                                   const int64_t *q_rows, const int64_t *keys, double *out,
+                                   int n_threads) {
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 64)
+#endif
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = index_score_fp8(q + (size_t)q_rows[i] * H * d, q_scale + (size_t)q_rows[i] * H,
+                             w + (size_t)q_rows[i] * H, k + (size_t)keys[i] * d,
+                             (double)k_scale[keys[i]], H, d);
+}
+
 /* Pair counts and FLOP counts ("DeepSeek DSA FLOPs": causal pair count,
  * selected pair count, full-prefix scoring and decode FLOPs). */
 OR_API double oracle_n_dense(double T) { return T * (T + 1.0) / 2.0; }

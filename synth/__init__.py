@@ -13,5 +13,7 @@ from .inputs import (  # noqa: F401
     make_decode,
     make_integer_prefill,
     make_prefill,
+    make_prefill_fp8,
+    quantize_e4m3_rows,
     random_distinct_keys,
 )

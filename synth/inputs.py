@@ -244,6 +244,35 @@ def make_prefill(wl: Workload | str, *, T_q: int | None = None, T_k: int | None 
     return out
 
 
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3_rows(bits: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """FP8 E4M3 codes and one fp32 scale per row of bf16 bit patterns (..., d).
+
+    scale = max|row| / 448 (1 for an all-zero row); codes = E4M3(value / scale)
+    rounded to nearest (torch's float8_e4m3fn conversion), so that the row's
+    largest magnitude maps to the largest finite code.
+    """
+    import torch
+    vals = bf16_bits_to_f32(bits).astype(np.float32)
+    amax = np.abs(vals).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    x = np.clip(vals / scale[..., None], -E4M3_MAX, E4M3_MAX).astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(x)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return codes, scale
+
+
+def make_prefill_fp8(wl: Workload | str, **kw) -> dict:
+    """make_prefill's inputs stored as FP8: q8 (T_q,H,d) and k8 (T_k,d) E4M3
+    codes with per-row fp32 scales q_scale (T_q,H) and k_scale (T_k,); the
+    bf16 inputs the codes were made from stay under q / k."""
+    x = make_prefill(wl, **kw)
+    x["q8"], x["q_scale"] = quantize_e4m3_rows(x["q"])
+    x["k8"], x["k_scale"] = quantize_e4m3_rows(x["k"])
+    return x
+
+
 def make_decode(wl: Workload | str, *, B: int | None = None, t_cap: int | None = None,
                 seq_len=None, seed: int | None = None) -> dict:
     """Generate B independent decode problems: q (B,H,d), w (B,H), k (B,t_cap,d).

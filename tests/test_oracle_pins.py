@@ -385,3 +385,51 @@ def test_score_pairs_agrees_with_the_chunk_and_decode_scores():
     for b in range(2):
         got = oracle.score_pairs(q[b:b + 1], w[b:b + 1], kc[b], np.zeros(5, np.int64), idx[b])
         assert (got == sc[b]).all()
+
+
+# ------------------------------------------------------------------ FP8 ----
+
+def test_e4m3_decode_matches_torch_float8():
+    # every FP8 E4M3 code decodes to the value a library routine gives
+    # (torch.float8_e4m3fn), NaN codes included
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert (got[~np.isnan(got)] == ref[~np.isnan(ref)]).all()
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+
+
+def test_fp8_scores_with_unit_scales_equal_the_bf16_scores():
+    # every E4M3 value is exactly a bf16 value, so with unit scales the FP8
+    # definition is the bf16 one on the same numbers
+    from synth import quantize_e4m3_rows
+    x = make_prefill("causal_16k_h64", T_q=12, T_k=300, q_offset=288, seed=5)
+    q8, _ = quantize_e4m3_rows(x["q"])
+    k8, _ = quantize_e4m3_rows(x["k"])
+    qb = bf16_bits_from_f64(oracle.e4m3_decode(q8).reshape(q8.shape))
+    kb = bf16_bits_from_f64(oracle.e4m3_decode(k8).reshape(k8.shape))
+    ones_q, ones_k = np.ones(q8.shape[:2], np.float32), np.ones(k8.shape[0], np.float32)
+    fi, fs, fa = oracle.prefill_topk_fp8(q8, ones_q, x["w"], k8, ones_k, 288, 40)
+    bi, bs, ba = oracle.prefill_topk(qb, x["w"], kb, 288, 40)
+    assert (fi == bi).all() and (fs == bs).all() and (fa == ba).all()
+
+
+def test_fp8_scales_act_as_positive_factors():
+    # a key scale multiplies every score of that key; a query head scale
+    # multiplies that head's weight (ReLU is positively homogeneous)
+    from synth import make_prefill_fp8
+    x = make_prefill_fp8("causal_16k_h64", T_q=4, T_k=64, q_offset=60, seed=6)
+    rows = np.repeat(np.arange(4), 64)
+    keys = np.tile(np.arange(64), 4)
+    base = oracle.score_pairs_fp8(x["q8"], x["q_scale"], x["w"], x["k8"], x["k_scale"], rows, keys)
+    ks2 = x["k_scale"] * np.float32(2.0)
+    assert np.allclose(oracle.score_pairs_fp8(x["q8"], x["q_scale"], x["w"], x["k8"], ks2, rows, keys),
+                       2.0 * base, rtol=1e-13, atol=0)
+    qs3, w3 = x["q_scale"].copy(), x["w"].copy()
+    qs3[:, 5] *= np.float32(4.0)
+    w3[:, 5] *= np.float32(4.0)
+    a = oracle.score_pairs_fp8(x["q8"], qs3, x["w"], x["k8"], x["k_scale"], rows, keys)
+    b = oracle.score_pairs_fp8(x["q8"], x["q_scale"], w3, x["k8"], x["k_scale"], rows, keys)
+    assert np.allclose(a, b, rtol=1e-13, atol=1e-300)
