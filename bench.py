@@ -36,7 +36,7 @@ import numpy as np
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
-from synth import WORKLOADS, make_decode, make_prefill  # noqa: E402
+from synth import WORKLOADS, make_decode, make_prefill, make_prefill_fp8  # noqa: E402
 
 DEFAULT_WORKLOAD = "causal_16k_h64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["dense", "pruned"], default="dense",
                     help="prefill path: dense fused scoring, or DoSA certified pruning")
+    ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="dense prefill inputs: bf16, or FP8 E4M3 codes with per-row scales")
     ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
                     help="N>1: independent replicas per rank (weak) or one workload split by rows (strong)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -160,7 +162,11 @@ def oracle_sample_rate(wl, x, target_s: float, rows_cap: int | None = None):
         def run(n):
             rows = np.unique(np.linspace(0, wl.T_q - 1, n).round().astype(np.int64))
             t0 = time.perf_counter()
-            oracle.prefill_topk(x["q"], x["w"], x["k"], x["q_offset"], wl.topk, rows=rows)
+            if "q8" in x:  # FP8 inputs: the FP8 oracle
+                oracle.prefill_topk_fp8(x["q8"], x["q_scale"], x["w"], x["k8"], x["k_scale"], x["q_offset"],
+                                        wl.topk, rows=rows)
+            else:
+                oracle.prefill_topk(x["q"], x["w"], x["k"], x["q_offset"], wl.topk, rows=rows)
             dt = time.perf_counter() - t0
             return dt, int((x["q_offset"] + rows + 1).sum()), len(rows)
         total_rows = wl.T_q
@@ -260,7 +266,12 @@ def main():
     pruned = args.path == "pruned"
     if pruned and (wl.kind != "prefill" or wl.n_seed == 0):
         raise SystemExit(f"--path pruned needs a chunked prefill workload with a seed set, not {wl.name}")
-    if wl.kind == "prefill":
+    fp8 = args.dtype == "fp8"
+    if fp8 and (wl.kind != "prefill" or pruned):
+        raise SystemExit("--dtype fp8 runs the dense prefill")
+    if fp8:
+        x = make_prefill_fp8(wl, seed=seed)
+    elif wl.kind == "prefill":
         x = make_prefill(wl, seed=seed, with_anchor=pruned)
     else:
         x = make_decode(wl, seed=seed)
@@ -279,6 +290,8 @@ def main():
         if e <= b:
             raise SystemExit(f"--shard rows: rank {rank} has no rows of {wl.name}")
         x["q"], x["w"] = x["q"][b:e], x["w"][b:e]
+        if fp8:
+            x["q8"], x["q_scale"] = x["q8"][b:e], x["q_scale"][b:e]
     else:
         pairs = wl.visible_pairs
     total_pairs = sum_over_ranks(pairs, dev) if world > 1 else pairs
@@ -327,6 +340,19 @@ def main():
             dsa.dsa_index_prefill_pruned(qq, ww, kk, q_off, wl.topk, seeds, out_idx=oi,
                                          out_score=osc, workspace=ws)
         n_kernels = 20  # launches of one pruned call (probe and rest of the chunk)
+    elif fp8:
+        ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(rows, wl.T_k, wl.H, wl.d, wl.topk),
+                         dtype=torch.uint8, device=dev)
+        q8 = torch.from_numpy(np.ascontiguousarray(x["q8"])).to(dev)
+        k8 = torch.from_numpy(np.ascontiguousarray(x["k8"])).to(dev)
+        qs = torch.from_numpy(x["q_scale"]).to(dev)
+        ks = torch.from_numpy(x["k_scale"]).to(dev)
+        del q, k
+
+        def step(qq=q8, ww=w, kk=k8, oi=out_idx, osc=out_score, qsc=qs, ksc=ks):
+            dsa.dsa_index_prefill_fp8(qq, qsc, ww, kk, ksc, q_off, wl.topk, out_idx=oi, out_score=osc,
+                                      workspace=ws)
+        n_kernels = 2
     elif wl.kind == "prefill":
         ws = torch.empty(dsa.dsa_index_prefill_workspace_bytes(rows, wl.T_k, wl.H, wl.d, wl.topk),
                          dtype=torch.uint8, device=dev)
@@ -413,9 +439,13 @@ def main():
     elif wl.kind == "prefill":
         flops = 2.0 * wl.H * wl.d * pairs
         achieved = flops / (score_ms * 1e-3) / 1e12
-        peak = float(pk["bf16_tflops"])
+        # FP8 takes its own dtype's peak: the measured bf16 burst figure times
+        # the nominal dense FP8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+        peak = float(pk["bf16_tflops"]) * (2.0 if fp8 else 1.0)
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"bf16_tflops (burst) of {pk_src}"}
+                "frac": achieved / peak,
+                "peak_source": (f"2 x bf16_tflops (burst) of {pk_src} (nominal fp8/bf16 ratio)" if fp8
+                                else f"bf16_tflops (burst) of {pk_src}")}
     else:
         nbytes = 2.0 * wl.d * pairs  # every visible key read once
         achieved = nbytes / (score_ms * 1e-3) / 1e9
@@ -427,12 +457,14 @@ def main():
         roof["kernel_ms"] = score_ms
         roof["traffic"] = recorded_traffic(wl.name, "score_topk_kernel")
     if roof["bound"] == "tensor":
-        # the same achieved rate against the other bf16 peaks: the sustained
-        # (power-capped) cuBLAS loop and the datasheet's dense figure
-        spec = 2250.0
-        roof["frac_vs_sustained"] = roof["achieved"] / float(pk["bf16_tflops_sustained"])
+        # the same achieved rate against the other peaks of the dtype: the
+        # sustained (power-capped) cuBLAS loop and the datasheet's dense figure
+        ratio = 2.0 if fp8 else 1.0
+        spec = 2250.0 * ratio
+        sus = float(pk["bf16_tflops_sustained"]) * ratio
+        roof["frac_vs_sustained"] = roof["achieved"] / sus
         roof["frac_vs_spec"] = roof["achieved"] / spec
-        roof["peaks_other"] = {"sustained": float(pk["bf16_tflops_sustained"]), "spec_dense_bf16": spec}
+        roof["peaks_other"] = {"sustained": sus, ("spec_dense_fp8" if fp8 else "spec_dense_bf16"): spec}
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -452,7 +484,26 @@ def main():
         d2h = hoi.numel() * 4 + hos.numel() * 4
         n_e2e = max(3, min(args.steps, 20))
         e_ms = []
-        if wl.kind == "prefill" and not pruned:
+        if fp8:
+            # FP8 codes and scales in, results out, on one stream
+            hq8 = torch.from_numpy(np.ascontiguousarray(x["q8"])).pin_memory()
+            hk8 = torch.from_numpy(np.ascontiguousarray(x["k8"])).pin_memory()
+            hqs, hks = torch.from_numpy(x["q_scale"]).pin_memory(), torch.from_numpy(x["k_scale"]).pin_memory()
+            dq8, dk8, dqs, dks, dw = (torch.empty_like(q8), torch.empty_like(k8), torch.empty_like(qs),
+                                      torch.empty_like(ks), torch.empty_like(w))
+            h2d = hq8.numel() + hk8.numel() + 4 * (hqs.numel() + hks.numel() + hw.numel())
+            e2e_api = "dsa_index_prefill_fp8: codes, scales and weights in, results out (one stream)"
+
+            def e2e_step():
+                dq8.copy_(hq8, non_blocking=True)
+                dk8.copy_(hk8, non_blocking=True)
+                dqs.copy_(hqs, non_blocking=True)
+                dks.copy_(hks, non_blocking=True)
+                dw.copy_(hw, non_blocking=True)
+                step(dq8, dw, dk8, out_idx, out_score, dqs, dks)
+                hoi.copy_(out_idx, non_blocking=True)
+                hos.copy_(out_score, non_blocking=True)
+        elif wl.kind == "prefill" and not pruned:
             # the library's host-buffer entry point: row blocks stream through
             # the device with the copies overlapping the kernels
             hws = torch.empty(dsa.dsa_index_prefill_host_workspace_bytes(rows, wl.T_k, wl.H, wl.d, wl.topk),
@@ -522,10 +573,10 @@ def main():
             "value": value, "unit": "pairs/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
+            "dtype": "fp8 (e4m3, fp32 scales)" if fp8 else "bf16", "data": "synthetic",
             "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
                            parallelism=(f"row blocks x{world}" if sharded else f"replicas x{world}"),
-                           path=args.path),
+                           path=args.path, inputs=args.dtype),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": n_kernels * args.steps, "clocks": clocks, "device_status": status,
             "kernel_ms": {n: float(np.mean(v)) for n, v in kern_ms.items()},

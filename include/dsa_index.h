@@ -84,13 +84,43 @@ DSA_API const char* dsa_last_error_string(void);
  *              q_offset + T_q <= T_k
  *   out_idx    device, [T_q][topk] int32
  *   out_score  device, [T_q][topk] fp32
- *   workspace  device, at least dsa_index_prefill_workspace_bytes() bytes
+ *   workspace  device, ws_bytes bytes.  dsa_index_prefill_workspace_bytes()
+ *              gives what one launch over all rows needs, capped at 4 GiB;
+ *              with less (at least one query group's worth, else
+ *              DSA_EWORKSPACE) the call runs consecutive launches over row
+ *              blocks that fit, with the same result bit for bit (rows are
+ *              independent).
  * T_q == 0 is a no-op.
  */
 DSA_API size_t dsa_index_prefill_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk);
 DSA_API int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
                       int64_t T_q, int64_t T_k, int H, int d, int topk, int32_t* out_idx,
                       float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The chunked causal prefill on FP8 inputs ("DeepSeek DSA FLOPs", Lightning
+ * Indexer: the indexer runs in FP8).  q and k are OCP FP8 E4M3 codes with one
+ * fp32 scale per stored row, so the vectors scored are
+ *     q(t,j) = q_scale[t][j] * e4m3(q[t][j]),   k(s) = k_scale[s] * e4m3(k[s]),
+ * and I(t,s) = sum_j w(t,j) * ReLU(q(t,j) . k(s)) as above.  Scales must be
+ * positive (or zero) and finite: they are applied as positive factors,
+ *     I(t,s) = k_scale[s] * sum_j (w(t,j) * q_scale[t][j]) * ReLU(e4m3 dot),
+ * the E4M3 dot products accumulating in fp32 on the tensor cores
+ * (tcgen05 kind::f8f6f4, products exact) and the head sum in the fp32 order
+ * stated above with halved weights w * q_scale / 2; a negative or non-finite
+ * key scale sets status bit 3.
+ *   q          device, [T_q][H][d] E4M3 codes (uint8), 16-byte aligned
+ *   q_scale    device, [T_q][H] fp32
+ *   w          device, [T_q][H] fp32
+ *   k          device, [T_k][d] E4M3 codes (uint8), 16-byte aligned
+ *   k_scale    device, [T_k] fp32
+ * Other arguments, outputs and the workspace (dsa_index_prefill_workspace_bytes)
+ * as for dsa_index_prefill; the same row-block rule applies.
+ */
+DSA_API int dsa_index_prefill_fp8(const uint8_t* q, const float* q_scale, const float* w, const uint8_t* k,
+                                  const float* k_scale, int64_t q_offset, int64_t T_q, int64_t T_k, int H,
+                                  int d, int topk, int32_t* out_idx, float* out_score, void* workspace,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * The same chunked causal prefill from HOST buffers: q, w and k are host

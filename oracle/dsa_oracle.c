@@ -478,13 +478,19 @@ OR_API void oracle_e4m3_decode(const uint8_t *codes, int64_t n, double *out) {
   for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_f64(codes[i]);
 }
 
+/* The 256 code values, filled from e4m3_to_f64 by the (serial) entry points
+ * before any parallel region reads it. */
+static double g_e4m3[256];
+static void e4m3_table(void) {
+  for (int c = 0; c < 256; ++c) g_e4m3[c] = e4m3_to_f64((uint8_t)c);
+}
+
 static double index_score_fp8(const uint8_t *q_row, const float *qs_row, const float *w_row,
                               const uint8_t *k_s, double ks, int H, int d) {
   double I = 0.0;
   for (int j = 0; j < H; ++j) {
     double x = 0.0, qs = (double)qs_row[j];
-    for (int i = 0; i < d; ++i)
-      x += (qs * e4m3_to_f64(q_row[(size_t)j * d + i])) * (ks * e4m3_to_f64(k_s[i]));
+    for (int i = 0; i < d; ++i) x += (qs * g_e4m3[q_row[(size_t)j * d + i]]) * (ks * g_e4m3[k_s[i]]);
     I += (double)w_row[j] * (x > 0.0 ? x : 0.0);
   }
   return I;
@@ -499,6 +505,7 @@ OR_API int oracle_prefill_topk_fp8(const uint8_t *q, const float *q_scale, const
   if (q_offset < 0 || q_offset + T_q > T_k || topk <= 0) return -1;
   for (int64_t i = 0; i < n_rows; ++i)
     if (rows[i] < 0 || rows[i] >= T_q) return -1;
+  e4m3_table();
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -527,6 +534,7 @@ OR_API void oracle_score_pairs_fp8(const uint8_t *q, const float *q_scale, const
                                    const uint8_t *k, const float *k_scale, int H, int d, int64_t n,
                                    const int64_t *q_rows, const int64_t *keys, double *out,
                                    int n_threads) {
+  e4m3_table();
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
 #pragma omp parallel for schedule(dynamic, 64)

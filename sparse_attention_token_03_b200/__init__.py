@@ -17,7 +17,7 @@ import torch
 from . import build as _build
 
 __all__ = [
-    "DSAError", "lib", "dsa_index_prefill", "dsa_index_decode",
+    "DSAError", "lib", "dsa_index_prefill", "dsa_index_prefill_fp8", "dsa_index_decode",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
     "dsa_index_decode_noalloc", "dsa_index_decode_noalloc_status", "dsa_index_prefill_pruned",
@@ -57,6 +57,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_prefill_workspace_bytes.restype = SZ
         L.dsa_index_prefill.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
         L.dsa_index_prefill.restype = I
+        L.dsa_index_prefill_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_prefill_fp8.restype = I
         L.dsa_index_prefill_host_workspace_bytes.argtypes = [I64, I64, I, I, I]
         L.dsa_index_prefill_host_workspace_bytes.restype = SZ
         L.dsa_index_prefill_host.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
@@ -160,6 +162,44 @@ def dsa_index_prefill(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_offse
                                        T_k, H, d, int(topk), out_idx.data_ptr(),
                                        out_score.data_ptr(), ws.data_ptr(), ws.numel(),
                                        _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def _codes(t: torch.Tensor, name: str, ndim: int, device) -> torch.Tensor:
+    """FP8 E4M3 codes given as uint8 or torch.float8_e4m3fn (viewed as uint8)."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    _need(t, name, torch.uint8, ndim, device)
+    return t
+
+
+def dsa_index_prefill_fp8(q: torch.Tensor, q_scale: torch.Tensor, w: torch.Tensor, k: torch.Tensor,
+                          k_scale: torch.Tensor, q_offset: int, topk: int, out_idx=None, out_score=None,
+                          workspace=None):
+    """Exact Top-k of the index score of a causal chunk on FP8 inputs.
+
+    q (T_q, H, d) and k (T_k, d) hold E4M3 codes (uint8 or float8_e4m3fn) with
+    fp32 scales q_scale (T_q, H) and k_scale (T_k,); w (T_q, H) fp32.  Returns
+    (out_idx, out_score) of shape (T_q, topk), as dsa_index_prefill.
+    """
+    dev = k.device
+    q = _codes(q, "q", 3, dev)
+    k = _codes(k, "k", 2, dev)
+    _need(q_scale, "q_scale", torch.float32, 2, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k_scale, "k_scale", torch.float32, 1, dev)
+    T_q, H, d = q.shape
+    T_k = k.shape[0]
+    if tuple(w.shape) != (T_q, H) or tuple(q_scale.shape) != (T_q, H) or k.shape[1] != d or \
+            k_scale.shape[0] != T_k:
+        raise ValueError("shape mismatch between q, q_scale, w, k and k_scale")
+    out_idx, out_score = _outputs(T_q, topk, dev, out_idx, out_score)
+    ws = _workspace(dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk), dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_fp8(q.data_ptr(), q_scale.data_ptr(), w.data_ptr(), k.data_ptr(),
+                                           k_scale.data_ptr(), int(q_offset), T_q, T_k, H, d, int(topk),
+                                           out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
+                                           ws.numel(), _stream_ptr(dev)))
     return out_idx, out_score
 
 

@@ -66,6 +66,22 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
   return DSA_OK;
 }
 
+// FP8 matrix [rows][128] of E4M3 codes read as tiles of box_rows x 128
+// codes (one 128-byte row each), 128B swizzle.
+int make_tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DSA_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ECUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
 int sm_count() {
   // per-device cache; host threads may race on it harmlessly (atomic, and
   // every writer stores the same value)
@@ -502,13 +518,26 @@ int check_prefill_args(int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d,
 // selection, on device buffers (arguments already checked).  reset_status
 // clears the workspace's device status word first; begin_profile starts the
 // per-kernel events, profile records them.
-int prefill_run(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset, int64_t T_q,
+// FP8 inputs of a prefill: the E4M3 codes and their per-row scales (q and k
+// of prefill_run then point at the codes).
+struct Fp8Scales {
+  const float* q_scale;  // [T_q][H]
+  const float* k_scale;  // [T_k]
+};
+
+int prefill_run(const void* q, const float* w, const void* k, int64_t q_offset, int64_t T_q,
                 int64_t T_k, int H, int topk, int32_t* out_idx, float* out_score, uint8_t* ws,
-                const PrefillPlan& P, bool reset_status, bool begin_profile, bool profile, cudaStream_t st) {
+                const PrefillPlan& P, bool reset_status, bool begin_profile, bool profile, cudaStream_t st,
+                const Fp8Scales* f8 = nullptr) {
   int rc;
   CUtensorMap tq, tk;
-  if ((rc = make_tmap(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
-  if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
+  if (f8) {
+    if ((rc = make_tmap_u8(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
+    if ((rc = make_tmap_u8(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
+  } else {
+    if ((rc = make_tmap(&tq, q, T_q * H, P.G * H)) != DSA_OK) return rc;
+    if ((rc = make_tmap(&tk, k, T_k, kTileKeys)) != DSA_OK) return rc;
+  }
   cudaError_t e;
   if (reset_status && (e = cudaMemsetAsync(ws, 0, 4, st)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   if (begin_profile) prof_begin(st);
@@ -527,7 +556,14 @@ int prefill_run(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_
   sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = reinterpret_cast<uint32_t*>(ws);
-  if ((e = launch_score(H, P.G, P.eg, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
+  if (f8) {
+    sp.q_scale = f8->q_scale;
+    sp.k_scale = f8->k_scale;
+    if ((e = launch_score_fp8(H, P.G, P.eg, tq, tk, sp, P.grid, st)) != cudaSuccess)
+      return cuda_fail(e, "FP8 score kernel launch");
+  } else if ((e = launch_score(H, P.G, P.eg, tq, tk, sp, P.grid, st)) != cudaSuccess) {
+    return cuda_fail(e, "score kernel launch");
+  }
   if (profile) prof_mark(st, "score_topk");
 
   SelectParams se{};
@@ -698,6 +734,35 @@ int dsa_index_prefill(const uint16_t* q, const float* w, const uint16_t* k, int6
     rc = prefill_run(q + static_cast<size_t>(r0) * H * kD, w + static_cast<size_t>(r0) * H, k, q_offset + r0, n,
                      T_k, H, topk, out_idx + static_cast<size_t>(r0) * topk, out_score + static_cast<size_t>(r0) * topk,
                      ws, P, r0 == 0, r0 == 0, true, st);
+    if (rc != DSA_OK) return rc;
+  }
+  return DSA_OK;
+}
+
+int dsa_index_prefill_fp8(const uint8_t* q, const float* q_scale, const float* w, const uint8_t* k,
+                          const float* k_scale, int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d, int topk,
+                          int32_t* out_idx, float* out_score, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_prefill_args(q_offset, T_q, T_k, H, d, topk);
+  if (rc != DSA_OK || T_q == 0) return rc;
+  if (!q || !q_scale || !w || !k || !k_scale || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(workspace, 16) || !aligned(w, 4) || !aligned(q_scale, 4) ||
+      !aligned(k_scale, 4) || !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k, workspace need 16 bytes)");
+  const int64_t br = prefill_block_rows(T_q, T_k, H, topk, ws_bytes);
+  if (br < 1)
+    return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes,
+                block_bytes(std::min<int64_t>(T_q, 256 / H), T_k, H, topk));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  for (int64_t r0 = 0; r0 < T_q; r0 += br) {
+    const int64_t n = std::min(br, T_q - r0);
+    const PrefillPlan P = plan_prefill(n, T_k, q_offset + r0, H, topk);
+    if (P.bytes > ws_bytes) return fail(DSA_EWORKSPACE, "internal: row block workspace too small");
+    const Fp8Scales f8{q_scale + static_cast<size_t>(r0) * H, k_scale};
+    rc = prefill_run(q + static_cast<size_t>(r0) * H * kD, w + static_cast<size_t>(r0) * H, k, q_offset + r0, n,
+                     T_k, H, topk, out_idx + static_cast<size_t>(r0) * topk, out_score + static_cast<size_t>(r0) * topk,
+                     ws, P, r0 == 0, r0 == 0, true, st, &f8);
     if (rc != DSA_OK) return rc;
   }
   return DSA_OK;

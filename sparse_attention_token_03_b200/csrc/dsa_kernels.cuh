@@ -141,6 +141,10 @@ struct ScoreParams {
   // wait_ns and the launch unwinds with the timeout bit
   int stall_loads;
   uint64_t wait_ns;         // limit of the pipeline waits (0: kWaitTimeoutNs)
+  // FP8 inputs: one positive fp32 scale per query head row [T_q][H] and per
+  // key [T_k] (the bf16 kernels ignore them)
+  const float* q_scale;
+  const float* k_scale;
   // refine: survivor key ids per row (stride surv_stride), the key matrix they
   // index, and an initial admission threshold record per row
   const int32_t* surv_ids;
@@ -198,12 +202,13 @@ struct DecodePlanParams {
 struct ScoreSmem {
   int n_cols;
   int ns;
-  int eg;   // epilogue warpgroups
-  int nqh;  // per-query score-code histograms (kHistBins bins each); 0 for the screen
+  int eg;    // epilogue warpgroups
+  int nqh;   // per-query score-code histograms (kHistBins bins each); 0 for the screen
+  int subs;  // 128-byte swizzled column blocks per row: 2 for bf16 (d = 128), 1 for FP8
   __host__ __device__ constexpr uint32_t q_sub() const { return static_cast<uint32_t>(n_cols) * 128u; }
-  __host__ __device__ constexpr uint32_t q_bytes() const { return 2u * q_sub(); }
+  __host__ __device__ constexpr uint32_t q_bytes() const { return static_cast<uint32_t>(subs) * q_sub(); }
   __host__ __device__ constexpr uint32_t k_sub() const { return 128u * 128u; }
-  __host__ __device__ constexpr uint32_t k_stage() const { return 2u * k_sub(); }
+  __host__ __device__ constexpr uint32_t k_stage() const { return static_cast<uint32_t>(subs) * k_sub(); }
   __host__ __device__ constexpr uint32_t off_k() const { return q_bytes(); }
   __host__ __device__ constexpr uint32_t off_w() const { return off_k() + ns * k_stage(); }
   // screening-plan scalars (screen) or the head weights of the tile's queries
@@ -233,6 +238,9 @@ void take_wait_injection(ScoreParams& p);
 // Launchers (defined in the .cu files).
 cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                          const ScoreParams& p, int grid, cudaStream_t stream);
+// The same fused kernel on FP8 (E4M3) query and key tiles (prefill only).
+cudaError_t launch_score_fp8(int H, int G, int eg, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                             const ScoreParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_screen(const CUtensorMap& tmap_plan, const CUtensorMap& tmap_k, const ScoreParams& p,
                           int grid, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);

@@ -261,20 +261,30 @@ __device__ __forceinline__ int cta_unit_step(const ScoreParams& p) {
   return tabled(p) ? 1 : static_cast<int>(gridDim.x);
 }
 
+// Head weight j of a query row as the epilogue uses it (before halving):
+// w for bf16 inputs; w times the row's scale for FP8 inputs (the query
+// scale is a positive factor of the head's ReLU term).
+template <bool F8>
+__device__ __forceinline__ float head_weight(const ScoreParams& p, int64_t i) {
+  if constexpr (F8) return __ldg(p.w + i) * __ldg(p.q_scale + i);
+  return __ldg(p.w + i);
+}
+
 }  // namespace
 
-template <int H, int G, int NS, int EG, int EPI>
+template <int H, int G, int NS, int EG, int EPI, bool F8 = false>
 __global__ void __launch_bounds__(score_threads(EG), 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams p) {
   constexpr int N = G * H;
   constexpr int GQ = G / EG;  // queries of a tile handled by one epilogue warpgroup
   constexpr bool kWSmem = EG >= 4;  // head weights read from shared memory (register budget)
-  constexpr ScoreSmem L{N, NS, EG, EPI == kEpiScore ? G : 0};
+  constexpr ScoreSmem L{N, NS, EG, EPI == kEpiScore ? G : 0, F8 ? 1 : 2};
   constexpr int ACC_COLS = N;
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32u : (2 * ACC_COLS <= 64) ? 64u
                                  : (2 * ACC_COLS <= 128) ? 128u : (2 * ACC_COLS <= 256) ? 256u : 512u;
-  constexpr uint32_t IDESC = idesc_bf16_f32(128, N);
+  constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N);
+  static_assert(!F8 || EPI == kEpiScore, "FP8 tiles feed the score epilogue only");
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
   static_assert(G % EG == 0, "queries must split evenly over the epilogue warpgroups");
 
@@ -332,7 +342,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   if (warp < score_epi_warp0(EG)) {
    // one setmaxnreg for the whole control warpgroup
    if constexpr (EG >= 2) regs_dec<regs_ctl(EG)>();
-   if (warp == 0 && p.mode == kModeRefine && !p.stall_loads) {
+   if (!F8 && warp == 0 && p.mode == kModeRefine && !p.stall_loads) {
     // ------------------------------------------------ producer (gathered keys)
     // Survivor keys are gathered row by row with 16-byte cp.async into the
     // 128B-swizzled layout the MMA reads.  A stage is signalled LAG tiles
@@ -403,8 +413,9 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         if (U.tile_hi <= U.tile_lo) continue;
         if (!(ok = mbar_wait(bar_q_empty, (qi & 1) ^ 1, s_abort, p.err, wlim))) break;
         mbar_arrive_expect_tx(bar_q_full, L.q_bytes());
+        // bf16: two 64-column boxes per row; FP8: one box of the 128 codes
         tma_load_2d(sQ, &tmap_q, 0, static_cast<int32_t>(U.q_row), bar_q_full);
-        tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
+        if constexpr (!F8) tma_load_2d(sQ + L.q_sub(), &tmap_q, 64, static_cast<int32_t>(U.q_row), bar_q_full);
         ++qi;
         if (u + u_step < u_end) {  // warm L2 with the next unit's query tile
           const Unit V = unit_geometry<G>(p, u + u_step, H);
@@ -417,7 +428,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           mbar_arrive_expect_tx(bar_k_full(s), L.k_stage());
           const int32_t krow = static_cast<int32_t>(U.k_row + t * kTileKeys);
           tma_load_2d(sK + s * L.k_stage(), &tmap_k, 0, krow, bar_k_full(s));
-          tma_load_2d(sK + s * L.k_stage() + L.k_sub(), &tmap_k, 64, krow, bar_k_full(s));
+          if constexpr (!F8) tma_load_2d(sK + s * L.k_stage() + L.k_sub(), &tmap_k, 64, krow, bar_k_full(s));
           ++kt;
         }
       }
@@ -449,11 +460,16 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           const uint32_t d_tmem = tmem_base + a * ACC_COLS;
           const uint32_t a_base = sK + s * L.k_stage();
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
+          // K steps of 32 bytes: 8 x (K = 16 bf16) or 4 x (K = 32 E4M3)
+          for (int kk = 0; kk < (F8 ? kD / 32 : kD / 16); ++kk) {
+            const uint32_t sub = F8 ? 0u : kk >> 2, off = (F8 ? kk : (kk & 3)) * 32;
             const uint64_t adesc = smem_desc_sw128(a_base + sub * L.k_sub() + off);
             const uint64_t bdesc = smem_desc_sw128(sQ + sub * L.q_sub() + off);
-            mma_bf16(d_tmem, adesc, bdesc, IDESC, kk > 0 ? 1u : 0u);
+            if constexpr (F8) {
+              mma_e4m3(d_tmem, adesc, bdesc, IDESC, kk > 0 ? 1u : 0u);
+            } else {
+              mma_bf16(d_tmem, adesc, bdesc, IDESC, kk > 0 ? 1u : 0u);
+            }
           }
           mma_commit(bar_k_empty(s));
           mma_commit(bar_acc_full(a));
@@ -597,7 +613,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         // this warpgroup's halved head weights, in shared memory for the whole unit
         for (int i = etid; i < GQ * H; i += kEpiThreads) {
           const int qq = q_lo + i / H;
-          s_w[q_lo * H + i] = qq < U.rows ? half_weight(__ldg(p.w + (U.row0 + qq) * H + i % H)) : 0.0f;
+          s_w[q_lo * H + i] = qq < U.rows ? half_weight(head_weight<F8>(p, (U.row0 + qq) * H + i % H)) : 0.0f;
         }
       }
       epi_sync(bar);
@@ -608,16 +624,10 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
-          const float4* src = reinterpret_cast<const float4*>(p.w + (U.row0 + (qq < U.rows ? qq : 0)) * H);
+          const int64_t wrow = (U.row0 + (qq < U.rows ? qq : 0)) * H;
+          const bool on = qq < U.rows;
 #pragma unroll
-          for (int j4 = 0; j4 < H / 4; ++j4) {
-            const float4 v = __ldg(src + j4);
-            const bool on = qq < U.rows;
-            wr[i][4 * j4 + 0] = on ? half_weight(v.x) : 0.0f;
-            wr[i][4 * j4 + 1] = on ? half_weight(v.y) : 0.0f;
-            wr[i][4 * j4 + 2] = on ? half_weight(v.z) : 0.0f;
-            wr[i][4 * j4 + 3] = on ? half_weight(v.w) : 0.0f;
-          }
+          for (int j = 0; j < H; ++j) wr[i][j] = on ? half_weight(head_weight<F8>(p, wrow + j)) : 0.0f;
         }
       }
       uint64_t* cand_unit = p.cand + static_cast<size_t>(U.slot) * G * lay.query_recs();
@@ -692,6 +702,13 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           }
         }
         ++at;
+        if constexpr (F8) {
+          // FP8: the key's scale multiplies its whole score (positive factor)
+          const float ks = key_local < p.T_k ? __ldg(p.k_scale + key_local) : 0.0f;
+          nonfinite = nonfinite || !(ks >= 0.0f && ks <= 3.402823466e38f);
+#pragma unroll
+          for (int i = 0; i < GQ; ++i) score[i] *= ks;
+        }
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
@@ -742,9 +759,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           // topk of them in bins >= B, a later key whose score code lies below
           // bin B is beaten by topk records and can never be selected.
           int kept_above = 0;
-          // (at the unit's last tile always: the final threshold goes to the
-          // unit's meta, where the final selection filters by it)
-          if (total >= p.topk && (full || total - s_upd[qq] >= 256 || t + 1 == U.tile_hi)) {
+          if (total >= p.topk && (full || total - s_upd[qq] >= 256)) {
             epi_find_bucket(qh, kHistBins, 0, p.topk, etid, s_misc + 4, s_misc + 1, bar);
             const uint64_t t_new = static_cast<uint64_t>(hist_edge(static_cast<uint32_t>(s_misc[1]))) << 32;
             kept_above = s_misc[2] + s_misc[3];
@@ -866,12 +881,12 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
-template <int H, int G, int NS, int EG, int EPI = kEpiScore>
+template <int H, int G, int NS, int EG, int EPI = kEpiScore, bool F8 = false>
 static cudaError_t launch_score_t(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const ScoreParams& p, int grid, cudaStream_t stream) {
-  constexpr ScoreSmem L{G * H, NS, EG, EPI == kEpiScore ? G : 0};
+  constexpr ScoreSmem L{G * H, NS, EG, EPI == kEpiScore ? G : 0, F8 ? 1 : 2};
   static_assert(L.request() <= 227u * 1024u, "shared memory budget");
-  auto kern = score_topk_kernel<H, G, NS, EG, EPI>;
+  auto kern = score_topk_kernel<H, G, NS, EG, EPI, F8>;
   int dev = 0;
   cudaGetDevice(&dev);
   // per (kernel instance, device); racing host threads only repeat the
@@ -905,6 +920,19 @@ cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tq, const CUte
   if (H == 32 && G == 8 && eg == 2) return launch_score_t<32, 8, 3, 2>(tq, tk, p, grid, stream);
   if (H == 64 && G == 1) return launch_score_t<64, 1, 6, 1>(tq, tk, p, grid, stream);
   if (H == 32 && G == 1) return launch_score_t<32, 1, 6, 1>(tq, tk, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_score_fp8(int H, int G, int eg, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const ScoreParams& p0, int grid, cudaStream_t stream) {
+  ScoreParams p = p0;
+  take_wait_injection(p);
+  if (p.mode != kModePrefill) return cudaErrorInvalidValue;
+  // FP8 stages are half the size: twice as many fit
+  if (H == 64 && G == 4 && eg == 4) return launch_score_t<64, 4, 8, 4, kEpiScore, true>(tq, tk, p, grid, stream);
+  if (H == 64 && G == 4 && eg == 2) return launch_score_t<64, 4, 8, 2, kEpiScore, true>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8 && eg == 4) return launch_score_t<32, 8, 6, 4, kEpiScore, true>(tq, tk, p, grid, stream);
+  if (H == 32 && G == 8 && eg == 2) return launch_score_t<32, 8, 6, 2, kEpiScore, true>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;
 }
 

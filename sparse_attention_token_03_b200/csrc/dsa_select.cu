@@ -278,24 +278,44 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
       }
     };
     if (table) {
-      const int nsg = n_seg;
-      for (int base = 0; base < total; base += kBatch * NT) {
-        uint64_t r[kBatch];
+      // thread tid reads the flattened indices tid, tid + NT, ...: its
+      // segment only moves forward; 8 streaming loads are in flight per step
+      constexpr int kLoads = 8;
+      int sg = 0;
+      for (int base = 0; base < total; base += kLoads * NT) {
+        uint64_t r[kLoads];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
+        for (int j = 0; j < kLoads; ++j) {
           const int i = base + j * NT + tid;
           r[j] = 0ull;
           if (i < total) {
-            int lo = 0, hi = nsg - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (s_segoff[mid] <= i) lo = mid; else hi = mid - 1;
-            }
-            r[j] = s_segptr[lo][i - s_segoff[lo]];
+            while (s_segoff[sg + 1] <= i) ++sg;
+            r[j] = __ldcs(reinterpret_cast<const unsigned long long*>(s_segptr[sg]) + (i - s_segoff[sg]));
           }
         }
+        // one shared-memory atomic per warp and step for the staging slots
+        uint32_t bal[kLoads];
+        int tot = 0;
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) take(base + j * NT + tid < total, r[j]);
+        for (int j = 0; j < kLoads; ++j) {
+          bal[j] = __ballot_sync(0xFFFFFFFFu, base + j * NT + tid < total && r[j] != 0ull && r[j] >= thr);
+          tot += __popc(bal[j]);
+        }
+        if (tot == 0) continue;
+        int at = 0;
+        if (lane == 0) at = atomicAdd(&s_n, tot);
+        at = __shfl_sync(0xFFFFFFFFu, at, 0);
+#pragma unroll
+        for (int j = 0; j < kLoads; ++j) {
+          if ((bal[j] >> lane) & 1u) {
+            const int pos = at + __popc(bal[j] & lanemask_lt());
+            if (pos < kSelStage) s_rec[pos] = r[j];
+            const uint32_t c = static_cast<uint32_t>(r[j] >> 32);
+            clo = min(clo, c);
+            chi = max(chi, c);
+          }
+          at += __popc(bal[j]);
+        }
       }
     } else {
       for (int sg = 0; sg < n_seg; ++sg) {
@@ -336,11 +356,13 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
     for (int i = tid; i < kSelBins; i += NT) s_hist[i] = 0u;
     // bucket of a record: linear in its score between the staged minimum and
     // maximum (any digit that never decreases along the record order keeps
-    // the selection exact; a linear one spreads the winners evenly), or, when
-    // that range is zero or not finite, the top 10 bits of (record - smallest)
+    // the selection exact; a linear one spreads the winners evenly, where the
+    // score code would crowd scores of both signs near zero), or, when that
+    // range is zero or not finite, the top 10 bits of (record - smallest)
     const float smin = record_score(s_lo), srange = record_score(s_hi) - smin;
     const float scale = static_cast<float>(kSelBins - 1) / srange;
     const bool lin = srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f;
+    __syncthreads();
     if (!lin) {
       uint64_t lo = ~0ull, hi = 0ull;
       for (int i = tid; i < n; i += NT) {
@@ -354,7 +376,6 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
         lo = l2 < lo ? l2 : lo;
         hi = h2 > hi ? h2 : hi;
       }
-      __syncthreads();
       if (tid == 0) {
         s_lo = ~0ull;
         s_hi = 0ull;
@@ -364,8 +385,8 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
         atomicMin(&s_lo, static_cast<unsigned long long>(lo));
         atomicMax(&s_hi, static_cast<unsigned long long>(hi));
       }
+      __syncthreads();
     }
-    __syncthreads();
     const uint64_t rlo = s_lo;
     const uint64_t span = s_hi - rlo;
     const int shift = max(0, 64 - __clzll(static_cast<long long>(span)) - 10);  // span >> shift < 1024
@@ -432,6 +453,7 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
+        if (j * NT >= n) break;
         if (v[j] == 0ull) continue;
         const uint32_t d = digit(v[j]);
         if (static_cast<int>(d) >= B) s_rec[atomicAdd(&s_cur[d], 1u)] = v[j];
