@@ -64,6 +64,8 @@ def _load():
                                                  P, P, P, I32]
         _lib.oracle_prefill_topk_fp8.restype = I32
         _lib.oracle_score_pairs_fp8.argtypes = [P, P, P, P, P, I32, I32, I64, P, P, P, I32]
+        _lib.oracle_seeds_from_history.argtypes = [P, I64, I32, I64, I32, P, P]
+        _lib.oracle_seeds_from_history.restype = I32
         for f in ("oracle_n_dense",):
             getattr(_lib, f).argtypes = [D]
             getattr(_lib, f).restype = D
@@ -184,6 +186,20 @@ def score_pairs_fp8(q, q_scale, w, k, k_scale, q_rows, keys, n_threads: int | No
     _load().oracle_score_pairs_fp8(_p(q), _p(q_scale), _p(w), _p(k), _p(k_scale), H, d, q_rows.shape[0],
                                    _p(q_rows), _p(keys), _p(out), n_threads or threads())
     return out
+
+
+def seeds_from_history(prev_idx, n_keys: int, n_seed: int):
+    """The n_seed keys below n_keys most often selected in prev_idx (rows of
+    earlier Top-k lists, -1 padding ignored), ties by the smaller key; returns
+    (seeds int32 in ascending key order, counts (n_keys,) int64)."""
+    prev = _c(prev_idx, np.int32)
+    n_rows, topk = prev.shape
+    seeds = np.empty(n_seed, np.int32)
+    counts = np.empty(n_keys, np.int64)
+    rc = _load().oracle_seeds_from_history(_p(prev), n_rows, topk, n_keys, n_seed, _p(seeds), _p(counts))
+    if rc != 0:
+        raise ValueError("oracle_seeds_from_history: bad arguments")
+    return seeds, counts
 
 
 def dosa_sample(seeds) -> np.ndarray:

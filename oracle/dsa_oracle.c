@@ -545,6 +545,48 @@ OR_API void oracle_score_pairs_fp8(const uint8_t *q, const float *q_scale, const
                              (double)k_scale[keys[i]], H, d);
 }
 
+/* ---------------------------------------------------------------------------
+ * Seeds from historical selection frequency (163.com write-up, section 03:
+ * seed candidates may be chosen by how often keys were selected before).
+ * Reading: count, over earlier query rows' Top-k lists prev[n_rows][topk]
+ * (-1 padding ignored), how many rows selected each key s < n_keys; the seeds
+ * are the n_seed keys with the largest counts, ties broken by the smaller
+ * key (keys never selected fill up from key 0), listed in ascending key order.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int64_t count;
+  int64_t key;
+} freq_t;
+
+static int freq_cmp(const void *pa, const void *pb) {
+  const freq_t *a = (const freq_t *)pa, *b = (const freq_t *)pb;
+  if (a->count != b->count) return a->count > b->count ? -1 : 1;
+  return (a->key < b->key) ? -1 : (a->key > b->key);
+}
+
+OR_API int oracle_seeds_from_history(const int32_t *prev, int64_t n_rows, int topk, int64_t n_keys,
+                                     int n_seed, int32_t *seeds, int64_t *counts_out) {
+  if (n_seed < 1 || n_seed > n_keys) return -1;
+  freq_t *f = (freq_t *)malloc(sizeof(freq_t) * (size_t)n_keys);
+  for (int64_t s = 0; s < n_keys; ++s) {
+    f[s].count = 0;
+    f[s].key = s;
+  }
+  for (int64_t i = 0; i < n_rows * topk; ++i)
+    if (prev[i] >= 0 && prev[i] < n_keys) f[prev[i]].count += 1;
+  if (counts_out)
+    for (int64_t s = 0; s < n_keys; ++s) counts_out[s] = f[s].count;
+  qsort(f, (size_t)n_keys, sizeof(freq_t), freq_cmp);
+  unsigned char *pick = (unsigned char *)calloc((size_t)n_keys, 1);
+  for (int i = 0; i < n_seed; ++i) pick[f[i].key] = 1;
+  int n = 0;
+  for (int64_t s = 0; s < n_keys; ++s)
+    if (pick[s]) seeds[n++] = (int32_t)s;
+  free(pick);
+  free(f);
+  return 0;
+}
+
 /* Pair counts and FLOP counts ("DeepSeek DSA FLOPs": causal pair count,
  * selected pair count, full-prefix scoring and decode FLOPs). */
 OR_API double oracle_n_dense(double T) { return T * (T + 1.0) / 2.0; }

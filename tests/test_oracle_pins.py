@@ -433,3 +433,32 @@ def test_fp8_scales_act_as_positive_factors():
     a = oracle.score_pairs_fp8(x["q8"], qs3, x["w"], x["k8"], x["k_scale"], rows, keys)
     b = oracle.score_pairs_fp8(x["q8"], x["q_scale"], w3, x["k8"], x["k_scale"], rows, keys)
     assert np.allclose(a, b, rtol=1e-13, atol=1e-300)
+
+
+# ------------------------------------------------------- history seeds ----
+
+def test_seeds_from_history_hand_example():
+    # 163.com write-up, section 03: seeds by historical selection frequency.
+    # Rows selected keys {5,2,7}, {2,7,-1}, {7,9,2}, {0,5,7}: counts
+    # 7:4, 2:3, 5:2, 0:1, 9:1, others 0; ties by the smaller key
+    prev = np.array([[5, 2, 7], [2, 7, -1], [7, 9, 2], [0, 5, 7]], np.int32)
+    # -> the seven most selected: 7, 2, 5, then 0 and 9 (count 1), then the
+    # never-selected 1 and 3; listed in ascending key order
+    seeds, counts = oracle.seeds_from_history(prev, 10, 7)
+    assert seeds.tolist() == [0, 1, 2, 3, 5, 7, 9]
+    assert counts.tolist() == [1, 0, 3, 0, 0, 2, 0, 4, 0, 1]
+    # keys at or beyond n_keys (not visible to the next chunk) never count
+    seeds, counts = oracle.seeds_from_history(prev, 6, 3)
+    assert seeds.tolist() == [0, 2, 5] and counts.tolist() == [1, 0, 3, 0, 0, 2]
+
+
+def test_seeds_from_history_properties():
+    # every chosen key was selected at least as often as every key left out,
+    # the seeds are distinct, and counts add up to the valid entries
+    rng = np.random.default_rng(4)
+    prev = rng.integers(-1, 400, size=(50, 16)).astype(np.int32)
+    seeds, counts = oracle.seeds_from_history(prev, 300, 64)
+    assert len(set(seeds.tolist())) == 64 and (seeds >= 0).all() and (seeds < 300).all()
+    out = np.setdiff1d(np.arange(300), seeds)
+    assert counts[seeds].min() >= counts[out].max()
+    assert counts.sum() == ((prev >= 0) & (prev < 300)).sum()
