@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--path", choices=["dense", "pruned"], default="dense",
                     help="prefill path: dense fused scoring, or DoSA certified pruning")
+    ap.add_argument("--paged", type=int, default=0,
+                    help="decode: keys in a shuffled page pool of this page size (a multiple of 64)")
     ap.add_argument("--dtype", choices=["bf16", "fp8"], default="bf16",
                     help="dense prefill inputs: bf16, or FP8 E4M3 codes with per-row scales")
     ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
@@ -361,6 +363,25 @@ def main():
             dsa.dsa_index_prefill(qq, ww, kk, q_off, wl.topk, out_idx=oi, out_score=osc,
                                   workspace=ws)
         n_kernels = 2
+    elif args.paged:
+        # the same caches scattered over a shuffled pool of pages
+        page = args.paged
+        B_, t_cap_ = x["k"].shape[0], x["k"].shape[1]
+        max_blocks = (t_cap_ + page - 1) // page
+        perm = np.random.default_rng(seed + 2).permutation(B_ * max_blocks).astype(np.int32)
+        bt = torch.from_numpy(perm.reshape(B_, max_blocks)).to(dev)
+        pool = torch.empty((B_ * max_blocks, page, wl.d), dtype=torch.bfloat16, device=dev)
+        kpad = torch.nn.functional.pad(k, (0, 0, 0, max_blocks * page - t_cap_))
+        pool[bt.reshape(-1).long()] = kpad.reshape(B_ * max_blocks, page, wl.d)
+        del kpad, k
+        k = pool
+        seq_len = torch.from_numpy(x["seq_len"]).to(dev)
+        ws = torch.empty(dsa.dsa_index_decode_workspace_bytes(rows, max_blocks * page, wl.H, wl.d, wl.topk),
+                         dtype=torch.uint8, device=dev)
+
+        def step(qq=q, ww=w, kk=pool, oi=out_idx, osc=out_score, sl=seq_len):
+            dsa.dsa_index_decode_paged(qq, ww, kk, bt, sl, wl.topk, out_idx=oi, out_score=osc, workspace=ws)
+        n_kernels = 3
     else:
         seq_len = torch.from_numpy(x["seq_len"]).to(dev)
         ws = torch.empty(dsa.dsa_index_decode_workspace_bytes(rows, wl.t_cap, wl.H, wl.d, wl.topk),
@@ -455,7 +476,7 @@ def main():
     if not pruned:
         roof["kernel"] = "score_topk_kernel"
         roof["kernel_ms"] = score_ms
-        roof["traffic"] = recorded_traffic(wl.name, "score_topk_kernel")
+        roof["traffic"] = recorded_traffic(wl.name + ("_fp8" if fp8 else ""), "score_topk_kernel")
     if roof["bound"] == "tensor":
         # the same achieved rate against the other peaks of the dtype: the
         # sustained (power-capped) cuBLAS loop and the datasheet's dense figure
@@ -468,7 +489,7 @@ def main():
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.paged:  # (the paged layout has no host-buffer leg)
         hq = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).view(torch.bfloat16).pin_memory()
         # (decode keeps its key cache on the device; the other paths take keys from the host)
         hk = (None if wl.kind == "decode" else
@@ -576,7 +597,8 @@ def main():
             "dtype": "fp8 (e4m3, fp32 scales)" if fp8 else "bf16", "data": "synthetic",
             "config": dict(workload_config(wl), l2="flushed between steps (256 MiB write)",
                            parallelism=(f"row blocks x{world}" if sharded else f"replicas x{world}"),
-                           path=args.path, inputs=args.dtype),
+                           path=args.path, inputs=args.dtype,
+                           **({"page_size": args.paged} if args.paged else {})),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": n_kernels * args.steps, "clocks": clocks, "device_status": status,
             "kernel_ms": {n: float(np.mean(v)) for n, v in kern_ms.items()},

@@ -69,6 +69,7 @@ typedef struct dsa_stats {
   int64_t records;        /* records written for the final selection (seed + refined) */
   int64_t recovered_rows; /* screened rows recomputed by the dense path (survivor overflow, bad seeds) */
   int64_t bypassed_rows;  /* rows the probe sent to the dense path without screening */
+  int64_t shared_keys;    /* keys of the groups' shared refine streams (each scored for 4 rows) */
 } dsa_stats;
 
 /* Text of the last error seen by this library in the calling thread. */
@@ -166,6 +167,28 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
                      void* stream);
 
 /*
+ * Batched decode over a PAGED key cache (the DoSA notes' port reads keys
+ * through pages, annotation LJZ23SXM; the layout here is this library's):
+ * sequence b's key i (0 <= i < seq_len[b]) is row
+ *     block_table[b][i / page_size] * page_size + i % page_size
+ * of the page pool.  Same computation and outputs as dsa_index_decode (key
+ * indices are positions within the sequence).
+ *   k_pages      device, [n_pages][page_size][d] bf16, 16-byte aligned
+ *   page_size    a positive multiple of 64
+ *   block_table  device, [B][max_blocks] int32 page ids; entries covering
+ *                keys below seq_len[b] must lie in [0, n_pages) (an entry
+ *                outside is read as page 0 and sets status bit 1)
+ *   seq_len      device, [B] int32, 0 <= seq_len[b] <= max_blocks * page_size
+ *                (a length outside is treated as 0 and sets status bit 1)
+ * The workspace is dsa_index_decode_workspace_bytes(B, max_blocks * page_size,
+ * ...).  Requires n_pages * page_size < 2^31.
+ */
+DSA_API int dsa_index_decode_paged(const uint16_t* q, const float* w, const uint16_t* k_pages, int64_t n_pages,
+                                   int page_size, const int32_t* block_table, int max_blocks,
+                                   const int32_t* seq_len, int B, int H, int d, int topk, int32_t* out_idx,
+                                   float* out_score, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Chunked causal prefill with DoSA certified pruning ("DoSA: Dots Sparse
  * Attention", steps 1-3; 163.com write-up, section 03).  Same inputs and the
  * same outputs, bit for bit, as dsa_index_prefill: the seed set only changes
@@ -178,6 +201,10 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
  *      U < tau are pruned (strictly; a key whose bound is uncertain is kept).
  *   3. Survivors are scored exactly with all heads; records at or above the
  *      row's topk-th seed record enter the final exact Top-k with the seeds'.
+ *      Within each group of four consecutive rows whose survivor lists all
+ *      fit, a key kept by at least two rows and visible to all four is
+ *      gathered once and scored for the four ("DoSA" notes, annotation
+ *      WFZZA9CL, step 3: the shared stream); the others are scored per row.
  * The first 64 rows of a chunk longer than 128 rows are a probe: they
  * always take steps 1-3, and from their survivor counts the device estimates
  * whether pruning pays for this chunk (screen, seed and refine costs against
@@ -198,8 +225,9 @@ DSA_API int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* 
  *              records: seed Top-k + refined candidates read by the final
  *              selection of the rows it finished; recovered_rows: screened
  *              rows recomputed densely after a survivor overflow or a bad
- *              seed list) and bypassed_rows (rows sent to the dense kernel
- *              without screening).
+ *              seed list), bypassed_rows (rows sent to the dense kernel
+ *              without screening) and shared_keys (keys of the shared
+ *              streams; refined_pairs counts four scores for each).
  * Requires T_q <= 65536.  The workspace is sized by
  * dsa_index_prefill_pruned_workspace_bytes().
  */
@@ -229,6 +257,31 @@ DSA_API int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_
                                                int64_t q_offset, int H, int d, int topk, int n_seed,
                                                uint32_t* mask, float* tau, int32_t* row_state,
                                                void* stream);
+
+/*
+ * Seed keys from historical selection frequency (163.com write-up, section
+ * 03: a chunk's seed set may be the keys that earlier rows selected most).
+ * Counts how often each key 0..n_keys-1 occurs in the Top-k lists of earlier
+ * rows and writes the n_seed keys with the largest counts, ties going to the
+ * smaller key (keys never selected fill up from key 0), in ascending key
+ * order.  With n_keys = the next chunk's q_offset and n_seed >= topk the
+ * output is a valid seed_idx for dsa_index_prefill_pruned.  Exact integer
+ * work; no host synchronisation.
+ *   prev_idx   device, [n_rows][topk] int32: earlier rows' out_idx; entries
+ *              outside [0, n_keys) (the -1 padding) are not counted.  May be
+ *              NULL when n_rows == 0 (then the seeds are keys 0..n_seed-1).
+ *   n_keys     1 <= n_keys < 2^31;  1 <= n_seed <= n_keys;
+ *              n_rows * topk < 2^32, else DSA_EINVAL.
+ *   seeds_out  device, [n_seed] int32, ascending.
+ *   workspace  device, 256-byte aligned, of
+ *              dsa_index_seeds_from_history_workspace_bytes(n_keys) bytes
+ *              (about 4 n_keys + 256 KB); after the call it holds the
+ *              per-key counts as uint32 at byte offset 256 + 262144.
+ */
+DSA_API size_t dsa_index_seeds_from_history_workspace_bytes(int64_t n_keys);
+DSA_API int dsa_index_seeds_from_history(const int32_t* prev_idx, int64_t n_rows, int topk, int64_t n_keys,
+                                         int n_seed, int32_t* seeds_out, void* workspace, size_t ws_bytes,
+                                         void* stream);
 
 /*
  * Batched decode that allocates nothing (no counterpart in the paper; a

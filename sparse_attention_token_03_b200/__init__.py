@@ -17,12 +17,13 @@ import torch
 from . import build as _build
 
 __all__ = [
-    "DSAError", "lib", "dsa_index_prefill", "dsa_index_prefill_fp8", "dsa_index_decode",
+    "DSAError", "lib", "dsa_index_prefill", "dsa_index_prefill_fp8", "dsa_index_decode", "dsa_index_decode_paged",
     "dsa_index_prefill_workspace_bytes", "dsa_index_decode_workspace_bytes",
     "dsa_index_device_status", "dsa_profile_enable", "dsa_profile_read",
     "dsa_index_decode_noalloc", "dsa_index_decode_noalloc_status", "dsa_index_prefill_pruned",
     "dsa_index_prefill_pruned_workspace_bytes", "dsa_index_prefill_pruned_survivors",
     "dsa_index_prefill_host", "dsa_index_prefill_host_workspace_bytes", "dsa_test_inject_wait_timeout",
+    "dsa_index_seeds_from_history", "dsa_index_seeds_from_history_workspace_bytes",
 ]
 
 DSA_OK = 0
@@ -67,12 +68,18 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_decode_workspace_bytes.restype = SZ
         L.dsa_index_decode.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]
         L.dsa_index_decode.restype = I
+        L.dsa_index_decode_paged.argtypes = [P, P, P, I64, I, P, I, P, I, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_decode_paged.restype = I
         L.dsa_index_prefill_pruned_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
         L.dsa_index_prefill_pruned_workspace_bytes.restype = SZ
         L.dsa_index_prefill_pruned.argtypes = [P, P, P, I64, I64, I64, I, I, I, P, I, P, P, P, P, SZ, P]
         L.dsa_index_prefill_pruned.restype = I
         L.dsa_index_prefill_pruned_survivors.argtypes = [P, I64, I64, I64, I, I, I, I, P, P, P, P]
         L.dsa_index_prefill_pruned_survivors.restype = I
+        L.dsa_index_seeds_from_history_workspace_bytes.argtypes = [I64]
+        L.dsa_index_seeds_from_history_workspace_bytes.restype = SZ
+        L.dsa_index_seeds_from_history.argtypes = [P, I64, I, I64, I, P, P, SZ, P]
+        L.dsa_index_seeds_from_history.restype = I
         L.dsa_index_decode_noalloc.argtypes = [P, P, P, P, I, I64, I, I, I, P, P, P]
         L.dsa_index_decode_noalloc.restype = I
         L.dsa_index_decode_noalloc_status.argtypes = [P, P]
@@ -256,7 +263,8 @@ def dsa_index_prefill_host(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, q_
 class _Stats(ctypes.Structure):
     _fields_ = [("screened_pairs", ctypes.c_int64), ("survivor_pairs", ctypes.c_int64),
                 ("refined_pairs", ctypes.c_int64), ("records", ctypes.c_int64),
-                ("recovered_rows", ctypes.c_int64), ("bypassed_rows", ctypes.c_int64)]
+                ("recovered_rows", ctypes.c_int64), ("bypassed_rows", ctypes.c_int64),
+                ("shared_keys", ctypes.c_int64)]
 
 
 def dsa_index_prefill_pruned_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int,
@@ -317,6 +325,34 @@ def dsa_index_prefill_pruned_survivors(workspace: torch.Tensor, T_q: int, T_k: i
     return mask, tau, state
 
 
+def dsa_index_seeds_from_history_workspace_bytes(n_keys: int) -> int:
+    return int(lib().dsa_index_seeds_from_history_workspace_bytes(int(n_keys)))
+
+
+def dsa_index_seeds_from_history(prev_idx: torch.Tensor, n_keys: int, n_seed: int, out=None, workspace=None):
+    """The n_seed keys below n_keys most often selected in prev_idx.
+
+    prev_idx (n_rows, topk) int32 on the GPU (earlier rows' out_idx, -1
+    padding ignored).  Returns (n_seed,) int32 in ascending key order: the
+    largest counts, ties to the smaller key.
+    """
+    dev = prev_idx.device
+    _need(prev_idx, "prev_idx", torch.int32, 2, dev)
+    n_rows, topk = prev_idx.shape
+    if out is None:
+        out = torch.empty(n_seed, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, 1, dev)
+    if out.shape[0] != n_seed:
+        raise ValueError(f"out must be ({n_seed},)")
+    nbytes = dsa_index_seeds_from_history_workspace_bytes(n_keys)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_seeds_from_history(prev_idx.data_ptr() if n_rows else None, n_rows, max(topk, 1),
+                                                  int(n_keys), int(n_seed), out.data_ptr(), ws.data_ptr(),
+                                                  ws.numel(), _stream_ptr(dev)))
+    return out
+
+
 def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
                      seq_len: torch.Tensor, topk: int, out_idx=None, out_score=None,
                      workspace=None):
@@ -342,6 +378,37 @@ def dsa_index_decode(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor,
                                       seq_len.data_ptr(), B, t_cap, H, d, int(topk),
                                       out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
                                       ws.numel(), _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_decode_paged(q: torch.Tensor, w: torch.Tensor, k_pages: torch.Tensor,
+                           block_table: torch.Tensor, seq_len: torch.Tensor, topk: int, out_idx=None,
+                           out_score=None, workspace=None):
+    """Exact Top-k for one new query per sequence against a paged key cache.
+
+    q (B, H, d) bf16, w (B, H) fp32, k_pages (n_pages, page_size, d) bf16 (the
+    page pool; page_size a multiple of 64), block_table (B, max_blocks) int32
+    page ids, seq_len (B,) int32.  Returns (out_idx, out_score) of shape
+    (B, topk) with key positions within each sequence.
+    """
+    dev = k_pages.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k_pages, "k_pages", torch.bfloat16, 3, dev)
+    _need(block_table, "block_table", torch.int32, 2, dev)
+    _need(seq_len, "seq_len", torch.int32, 1, dev)
+    B, H, d = q.shape
+    n_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    max_blocks = block_table.shape[1]
+    if tuple(w.shape) != (B, H) or k_pages.shape[2] != d or block_table.shape[0] != B or seq_len.shape[0] != B:
+        raise ValueError("shape mismatch between q, w, k_pages, block_table and seq_len")
+    out_idx, out_score = _outputs(B, topk, dev, out_idx, out_score)
+    ws = _workspace(dsa_index_decode_workspace_bytes(B, max_blocks * page_size, H, d, topk), dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_decode_paged(q.data_ptr(), w.data_ptr(), k_pages.data_ptr(), n_pages, page_size,
+                                            block_table.data_ptr(), max_blocks, seq_len.data_ptr(), B, H, d,
+                                            int(topk), out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(),
+                                            ws.numel(), _stream_ptr(dev)))
     return out_idx, out_score
 
 

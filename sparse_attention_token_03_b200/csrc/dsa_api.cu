@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -80,6 +81,28 @@ int make_tmap_u8(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DSA_ECUDA, "cuTensorMapEncodeTiled (u8) failed (%d)", static_cast<int>(r));
   return DSA_OK;
+}
+
+// Workspace of dsa_index_seeds_from_history: status word, control words,
+// count histogram and counts (one memset clears all four), tile prefixes.
+struct HistoryPlan {
+  size_t off_ctl, off_hist, off_counts, off_tile_gt, off_tile_eq, zero_bytes, bytes;
+};
+
+HistoryPlan plan_history(int64_t n_keys) {
+  HistoryPlan P{};
+  const size_t n_tiles = static_cast<size_t>((n_keys + 1023) / 1024);
+  P.off_ctl = 64;
+  P.off_hist = 256;
+  P.off_counts = P.off_hist + 65536 * 4;
+  size_t off = P.off_counts + static_cast<size_t>(n_keys) * 4;
+  P.zero_bytes = off;
+  off = (off + 255) / 256 * 256;
+  P.off_tile_gt = off;
+  off = (off + n_tiles * 4 + 255) / 256 * 256;
+  P.off_tile_eq = off;
+  P.bytes = (off + n_tiles * 4 + 255) / 256 * 256;
+  return P;
 }
 
 int sm_count() {
@@ -201,7 +224,9 @@ struct DecodePlan {
 constexpr size_t align_c(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout of a batched decode of B sequences run on `grid` CTAs.
-constexpr DecodePlan plan_decode_layout(int B, int topk, int grid) {
+// (g_rows > 1: each unit scores g_rows consecutive rows, the shared refine
+// stream's groups)
+constexpr DecodePlan plan_decode_layout(int B, int topk, int grid, int g_rows = 1) {
   DecodePlan P{};
   P.grid = grid;
   P.units_max = P.grid + B;
@@ -218,9 +243,9 @@ constexpr DecodePlan plan_decode_layout(int B, int topk, int grid) {
   P.off_seq_ucnt = off;
   off = align_c(off + static_cast<size_t>(B) * sizeof(int32_t), 256);
   P.off_meta = off;
-  off = align_c(off + static_cast<size_t>(P.units_max) * kMetaInts * sizeof(int32_t), 256);
+  off = align_c(off + static_cast<size_t>(P.units_max) * g_rows * kMetaInts * sizeof(int32_t), 256);
   P.off_cand = off;
-  off = align_c(off + static_cast<size_t>(P.units_max) * P.lay.query_recs() * sizeof(uint64_t), 256);
+  off = align_c(off + static_cast<size_t>(P.units_max) * g_rows * P.lay.query_recs() * sizeof(uint64_t), 256);
   P.bytes = off;
   return P;
 }
@@ -245,14 +270,30 @@ int check_decode_args(const uint16_t* q, const float* w, const uint16_t* k_cache
 
 // The decode path proper (arguments already validated): planner, fused score
 // kernel and final selection, all on `st`, scratch in `ws` laid out by P.
+// A paged key cache: the page pool [n_pages][page_size][128] and the
+// sequences' block tables [B][max_blocks].
+struct PagedKeys {
+  const int32_t* block_table;
+  int max_blocks;
+  int page_size;
+  int64_t n_pages;
+};
+
 int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const int32_t* seq_len,
                int B, int64_t t_cap, int H, int topk, int32_t* out_idx, float* out_score,
-               uint8_t* ws, const DecodePlan& P, bool profile, cudaStream_t st) {
+               uint8_t* ws, const DecodePlan& P, bool profile, cudaStream_t st, const PagedKeys* paged = nullptr) {
   int rc;
   CUtensorMap tq, tk;
   if ((rc = make_tmap(&tq, q, static_cast<int64_t>(B) * H, H)) != DSA_OK) return rc;
-  if ((rc = make_tmap(&tk, k_cache, std::max<int64_t>(static_cast<int64_t>(B) * t_cap, 1), kTileKeys)) != DSA_OK)
+  if (paged) {
+    // pages of a multiple of 128 keys hold whole key tiles (128-row boxes);
+    // 64-key pages split a tile's halves over two pages (64-row boxes)
+    const int box = paged->page_size % kTileKeys == 0 ? kTileKeys : 64;
+    if ((rc = make_tmap(&tk, k_cache, paged->n_pages * paged->page_size, box)) != DSA_OK) return rc;
+  } else if ((rc = make_tmap(&tk, k_cache, std::max<int64_t>(static_cast<int64_t>(B) * t_cap, 1), kTileKeys)) !=
+             DSA_OK) {
     return rc;
+  }
   cudaError_t e = cudaMemsetAsync(ws, 0, 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   if (profile) prof_begin(st);
@@ -284,6 +325,12 @@ int decode_run(const uint16_t* q, const float* w, const uint16_t* k_cache, const
   sp.cand = reinterpret_cast<uint64_t*>(ws + P.off_cand);
   sp.meta = reinterpret_cast<int32_t*>(ws + P.off_meta);
   sp.err = dp.err;
+  if (paged) {
+    sp.block_table = paged->block_table;
+    sp.max_blocks = paged->max_blocks;
+    sp.page_size = paged->page_size;
+    sp.n_pages = paged->n_pages;
+  }
   if ((e = launch_score(H, 1, 1, tq, tk, sp, P.grid, st)) != cudaSuccess) return cuda_fail(e, "score kernel launch");
   if (profile) prof_mark(st, "score_topk");
 
@@ -323,12 +370,14 @@ struct PrunedPlan {
   PrefillPlan screen[2];  // screening geometry (16 plan rows per query), same split
   PrefillPlan dense;      // exact dense pass over flagged rows
   DecodePlan refine;      // refine: one "sequence" of survivors per row
+  DecodePlan refine2;     // shared refine stream: one "sequence" per group of four rows
+  int64_t n_groups;
   int cap_row;            // survivor ids kept per row
   int rec_stride;         // seed records per row (topk rounded up to even)
   int64_t mask_words;
   size_t off_stats, off_ctl, off_seed_bits, off_k_seed, off_cand, off_seed_rec, off_tau, off_plan_q, off_plan_s,
       off_knorm, off_bitmask, off_surv_count, off_surv_ids, off_refine_len, off_row_flags, off_init_thr,
-      off_refine, bytes;
+      off_refine, off_group_mask, off_group_ids, off_group_len, off_refine2, bytes;
 };
 
 int pruned_cap_row(int64_t T_k, int topk) {
@@ -350,6 +399,8 @@ PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int to
   }
   P.dense = plan_prefill(T_q, T_k, q_offset, H, topk);
   P.refine = plan_decode(static_cast<int>(T_q), topk);
+  P.n_groups = (T_q + 3) / 4;
+  P.refine2 = plan_decode_layout(static_cast<int>(P.n_groups), topk, std::min(sm_count(), 1024), 4);
   P.cap_row = pruned_cap_row(T_k, topk);
   P.rec_stride = (topk + 1) & ~1;
   P.mask_words = (T_k + 31) / 32;
@@ -377,6 +428,10 @@ PrunedPlan plan_pruned(int64_t T_q, int64_t T_k, int64_t q_offset, int H, int to
   P.off_row_flags = take(static_cast<size_t>(T_q) * 4);
   P.off_init_thr = take(static_cast<size_t>(T_q) * 8);
   P.off_refine = take(P.refine.bytes);
+  P.off_group_mask = take(static_cast<size_t>(P.n_groups) * P.mask_words * 4);
+  P.off_group_ids = take(static_cast<size_t>(P.n_groups) * P.cap_row * 4);
+  P.off_group_len = take(static_cast<size_t>(P.n_groups) * 4);
+  P.off_refine2 = take(P.refine2.bytes);
   P.bytes = off;
   return P;
 }
@@ -466,12 +521,20 @@ int pruned_rows(const PrunedPlan& P, int i, int64_t r0, int64_t n, const uint16_
   s3.skip = skip;
   if ((e = launch_screen(tplan, tk, s3, CP.grid, st)) != cudaSuccess) return cuda_fail(e, "screen launch");
   prof_mark(st, "screen");
-  // survivors -> id lists; rows whose survivors overflow are flagged
+  // the shared refine stream of every full group of four rows (r0 is a
+  // multiple of four), then the rows' own id lists without those keys; rows
+  // whose survivors overflow are flagged
+  uint32_t* gmask = reinterpret_cast<uint32_t*>(at(P.off_group_mask)) + (r0 / 4) * P.mask_words;
+  int32_t* glen = reinterpret_cast<int32_t*>(at(P.off_group_len)) + r0 / 4;
+  ShareParams sh{n, q_offset + r0, bitmask, P.mask_words, surv_count, P.cap_row, gmask,
+                 reinterpret_cast<int32_t*>(at(P.off_group_ids)) + (r0 / 4) * P.cap_row, glen, err, skip};
+  if ((e = launch_share(sh, st)) != cudaSuccess) return cuda_fail(e, "share launch");
+  prof_mark(st, "share");
   CompactParams cp{n, q_offset + r0, topk, bitmask, P.mask_words, surv_count, P.cap_row,
                    reinterpret_cast<int32_t*>(at(P.off_surv_ids)) + r0 * P.cap_row,
                    reinterpret_cast<int32_t*>(at(P.off_refine_len)) + r0,
                    reinterpret_cast<int32_t*>(at(P.off_row_flags)) + r0, seed_rec, P.rec_stride,
-                   reinterpret_cast<uint64_t*>(at(P.off_init_thr)) + r0, err, skip};
+                   reinterpret_cast<uint64_t*>(at(P.off_init_thr)) + r0, err, skip, gmask, glen};
   if ((e = launch_compact(cp, st)) != cudaSuccess) return cuda_fail(e, "compact launch");
   prof_mark(st, "compact");
   return DSA_OK;
@@ -857,6 +920,30 @@ int dsa_index_decode(const uint16_t* q, const float* w, const uint16_t* k_cache,
                     static_cast<uint8_t*>(workspace), P, true, static_cast<cudaStream_t>(stream));
 }
 
+int dsa_index_decode_paged(const uint16_t* q, const float* w, const uint16_t* k_pages, int64_t n_pages,
+                           int page_size, const int32_t* block_table, int max_blocks, const int32_t* seq_len, int B,
+                           int H, int d, int topk, int32_t* out_idx, float* out_score, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  if (page_size < 64 || page_size % 64 != 0 || max_blocks < 1 || n_pages < 1)
+    return fail(DSA_EINVAL, "need page_size a positive multiple of 64, max_blocks >= 1, n_pages >= 1");
+  if (n_pages * page_size >= (int64_t(1) << 31)) return fail(DSA_EINVAL, "n_pages * page_size must be below 2^31");
+  const int64_t t_cap = static_cast<int64_t>(max_blocks) * page_size;
+  int rc = check_shape(H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if (B < 1 || B > 65536) return fail(DSA_EINVAL, "need 1 <= B <= 65536");
+  if (t_cap >= (int64_t(1) << 31)) return fail(DSA_EINVAL, "max_blocks * page_size must be below 2^31");
+  if (!q || !w || !k_pages || !block_table || !seq_len || !out_idx || !out_score || !workspace)
+    return fail(DSA_EINVAL, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(workspace, 16) || !aligned(w, 4) ||
+      !aligned(block_table, 4) || !aligned(seq_len, 4) || !aligned(out_idx, 4) || !aligned(out_score, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (q, k_pages and workspace need 16 bytes)");
+  const DecodePlan P = plan_decode(B, topk);
+  if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
+  const PagedKeys pk{block_table, max_blocks, page_size, n_pages};
+  return decode_run(q, w, k_pages, seq_len, B, t_cap, H, topk, out_idx, out_score, static_cast<uint8_t*>(workspace),
+                    P, true, static_cast<cudaStream_t>(stream), &pk);
+}
+
 int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* k, int64_t q_offset,
                              int64_t T_q, int64_t T_k, int H, int d, int topk, const int32_t* seed_idx,
                              int n_seed, int32_t* out_idx, float* out_score, dsa_stats* stats,
@@ -894,7 +981,8 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
   if ((e = cudaMemsetAsync(at(P.off_stats), 0, 8 * sizeof(unsigned long long), st)) != cudaSuccess ||
       (e = cudaMemsetAsync(bypass, 0, 8 * sizeof(uint32_t), st)) != cudaSuccess ||
       (e = cudaMemsetAsync(at(P.off_seed_bits), 0, P.mask_words * 4, st)) != cudaSuccess ||
-      (e = cudaMemsetAsync(surv_count, 0, T_q * 4, st)) != cudaSuccess)
+      (e = cudaMemsetAsync(surv_count, 0, T_q * 4, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(at(P.off_group_len), 0, P.n_groups * 4, st)) != cudaSuccess)
     return cuda_fail(e, "cudaMemsetAsync");
   prof_begin(st);
 
@@ -958,6 +1046,35 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
   s4.init_thr = reinterpret_cast<const uint64_t*>(at(P.off_init_thr));
   if ((e = launch_score(H, 1, 1, tqrow, tk, s4, R.grid, st)) != cudaSuccess) return cuda_fail(e, "refine launch");
   prof_mark(st, "refine");
+  // the shared stream: each group's shared keys scored once for its four rows
+  uint8_t* rws2 = at(P.off_refine2);
+  const DecodePlan& R2 = P.refine2;
+  DecodePlanParams dq2{};
+  dq2.B = static_cast<int>(P.n_groups);
+  dq2.grid = R2.grid;
+  dq2.t_cap = P.cap_row;
+  dq2.seq_len = reinterpret_cast<const int32_t*>(at(P.off_group_len));
+  dq2.seq_start = reinterpret_cast<int64_t*>(rws2 + R2.off_seq_start);
+  dq2.unit_tab = reinterpret_cast<int32_t*>(rws2 + R2.off_unit_tab);
+  dq2.cta_ubeg = reinterpret_cast<int32_t*>(rws2 + R2.off_cta_ubeg);
+  dq2.seq_ubeg = reinterpret_cast<int32_t*>(rws2 + R2.off_seq_ubeg);
+  dq2.seq_ucnt = reinterpret_cast<int32_t*>(rws2 + R2.off_seq_ucnt);
+  dq2.err = err;
+  if ((e = launch_decode_plan(dq2, st)) != cudaSuccess) return cuda_fail(e, "shared refine plan launch");
+  CUtensorMap tq4;
+  if ((rc = make_tmap(&tq4, q, T_q * H, 4 * H)) != DSA_OK) return rc;
+  ScoreParams s4b = s4;
+  s4b.mode = kModeRefineShared;
+  s4b.T_q = T_q;
+  s4b.seq_len = dq2.seq_len;
+  s4b.unit_tab = dq2.unit_tab;
+  s4b.cta_ubeg = dq2.cta_ubeg;
+  s4b.cand = reinterpret_cast<uint64_t*>(rws2 + R2.off_cand);
+  s4b.meta = reinterpret_cast<int32_t*>(rws2 + R2.off_meta);
+  s4b.surv_ids = reinterpret_cast<const int32_t*>(at(P.off_group_ids));
+  if ((e = launch_refine_shared(H, tq4, tk, s4b, R2.grid, st)) != cudaSuccess)
+    return cuda_fail(e, "shared refine launch");
+  prof_mark(st, "refine_shared");
   SelectParams s5{};
   s5.mode = kModeDecode;
   s5.G = 1;
@@ -969,6 +1086,11 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
   s5.meta = s4.meta;
   s5.seq_ubeg = dq.seq_ubeg;
   s5.seq_ucnt = dq.seq_ucnt;
+  s5.cand2 = s4b.cand;
+  s5.meta2 = s4b.meta;
+  s5.ubeg2 = dq2.seq_ubeg;
+  s5.ucnt2 = dq2.seq_ucnt;
+  s5.G2 = 4;
   s5.extra_rec = reinterpret_cast<const uint64_t*>(at(P.off_seed_rec));
   s5.rec_stride = P.rec_stride;
   s5.row_flags = row_flags;
@@ -1019,7 +1141,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
   if (stats) {
     unsigned long long* cnt = reinterpret_cast<unsigned long long*>(at(P.off_stats));
     StatsParams sp{T_q, q_offset, n_seed, topk, R.lay, surv_count, refine_len, row_flags, s4.meta,
-                   dq.seq_ubeg, dq.seq_ucnt, cnt};
+                   dq.seq_ubeg, dq.seq_ucnt, dq2.seq_len, s4b.meta, dq2.seq_ubeg, dq2.seq_ucnt, cnt};
     if ((e = launch_stats(sp, st)) != cudaSuccess) return cuda_fail(e, "stats launch");
     unsigned long long h[8] = {};
     uint32_t status = 0;
@@ -1033,6 +1155,7 @@ int dsa_index_prefill_pruned(const uint16_t* q, const float* w, const uint16_t* 
     stats->bypassed_rows = static_cast<int64_t>(h[3]);
     stats->screened_pairs = static_cast<int64_t>(h[4]);
     stats->records = static_cast<int64_t>(h[5]);
+    stats->shared_keys = static_cast<int64_t>(h[6]);
     if (status & kErrSeed) return fail(DSA_ESEED, "a seed was out of range or repeated; the rows were recomputed densely");
     if (status & kErrTimeout) return fail(DSA_EDEVICE, "a device-side wait gave up (status 0x%x)", status);
     if (status & kErrNonFinite) return fail(DSA_EDEVICE, "a visible pair scored inf or NaN (non-finite input)");
@@ -1059,6 +1182,46 @@ int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_q, int64
       (e = cudaMemcpyAsync(row_state, ws + P.off_row_flags, static_cast<size_t>(T_q) * 4, cudaMemcpyDeviceToDevice,
                            st)) != cudaSuccess)
     return cuda_fail(e, "copying the screen's survivor mask");
+  return DSA_OK;
+}
+
+size_t dsa_index_seeds_from_history_workspace_bytes(int64_t n_keys) {
+  if (n_keys < 1 || n_keys > INT32_MAX) return 0;
+  return plan_history(n_keys).bytes;
+}
+
+int dsa_index_seeds_from_history(const int32_t* prev_idx, int64_t n_rows, int topk, int64_t n_keys, int n_seed,
+                                 int32_t* seeds_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!seeds_out || !workspace || (n_rows > 0 && !prev_idx)) return fail(DSA_EINVAL, "null pointer argument");
+  if (n_rows < 0 || topk < 1 || n_keys < 1 || n_keys > INT32_MAX)
+    return fail(DSA_EINVAL, "n_rows = %lld, topk = %d, n_keys = %lld: need n_rows >= 0, topk >= 1, 1 <= n_keys < 2^31",
+                static_cast<long long>(n_rows), topk, static_cast<long long>(n_keys));
+  if (n_seed < 1 || n_seed > n_keys)
+    return fail(DSA_EINVAL, "n_seed = %d outside [1, n_keys = %lld]", n_seed, static_cast<long long>(n_keys));
+  if (n_rows > 0 && n_rows > static_cast<int64_t>(UINT32_MAX) / topk)
+    return fail(DSA_EINVAL, "n_rows * topk = %lld * %d exceeds 2^32 - 1 list entries",
+                static_cast<long long>(n_rows), topk);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return fail(DSA_EINVAL, "workspace not 256-byte aligned");
+  const HistoryPlan P = plan_history(n_keys);
+  if (ws_bytes < P.bytes) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, P.bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, P.zero_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  HistoryParams hp{};
+  hp.prev = prev_idx;
+  hp.n_rows = n_rows;
+  hp.topk = topk;
+  hp.n_keys = n_keys;
+  hp.n_seed = n_seed;
+  hp.num_sms = sm_count();
+  hp.counts = reinterpret_cast<uint32_t*>(ws + P.off_counts);
+  hp.hist = reinterpret_cast<uint32_t*>(ws + P.off_hist);
+  hp.ctl = reinterpret_cast<uint32_t*>(ws + P.off_ctl);
+  hp.tile_gt = reinterpret_cast<uint32_t*>(ws + P.off_tile_gt);
+  hp.tile_eq = reinterpret_cast<uint32_t*>(ws + P.off_tile_eq);
+  hp.seeds = seeds_out;
+  if ((e = launch_history_seeds(hp, st)) != cudaSuccess) return cuda_fail(e, "history seed kernels");
   return DSA_OK;
 }
 

@@ -96,12 +96,16 @@ __global__ void keynorm_kernel(const uint16_t* __restrict__ k, int64_t T_k, floa
 //               coefficients keep the bound valid), rho_j = ||q_j - sum c q_i||
 //  alpha_i = sum_P w_j |c_ji|,  beta = sum_P w_j rho_j
 //  q_pos = sum_P w_j q_j, q_neg = sum_N |w_j| q_j (rounded to bf16 for the MMA)
-// With d = q . k, the screening bound (see the screen epilogue) is
-//  U = sum_R [w_i max(d_i,0) + alpha_i |d_i| / 2] + d_pos/2 - max(d_neg,0) + C ||k||
-//  C = beta/2 + ||q_pos - bf16(q_pos)||/2 + ||q_neg - bf16(q_neg)|| + 2^-10 S,
+// With d = q . k, the screening bound is
+//  U = sum_R [w_i max(d_i,0) + alpha_i |d_i| / 2] + d_pos/2 - max(d_neg,0) + C ||k||,
+// evaluated (w max(d,0) = w d/2 + w |d|/2) as
+//  U = L . k + sum_R c_i |d_i| - max(d_neg,0) + C ||k||,
+//  L = q_pos/2 + sum_R (w_i/2) q_i,   c_i = (w_i + alpha_i)/2,
+//  C = beta/2 + ||L - bf16(L)|| + ||q_neg - bf16(q_neg)|| + 2^-10 S,
 //  S = sum_j |w_j| ||q_j|| + ||q_pos|| + ||q_neg|| + sum_R alpha_i ||q_i||,
 // where the last term absorbs the fp32 tensor-core accumulation and the fp32
 // arithmetic of the bound and of the exact score (each far below 2^-10 S ||k||).
+// Plan rows: the retained q_i, then L, then q_neg (bf16).
 // ---------------------------------------------------------------------------
 template <int H>
 __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
@@ -294,7 +298,10 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
   }
   __syncthreads();
 
-  // folded auxiliary rows (thread e owns element e), in ascending head order
+  // folded auxiliary rows (thread e owns element e), in ascending head
+  // order: the positive omitted heads' q_pos, the negative ones' q_neg, and
+  // the linear row L = q_pos / 2 + sum_R (w_i / 2) q_i, which carries the
+  // linear half of the bound (w max(d, 0) = w d / 2 + w |d| / 2) into the MMA
   {
     const int e = tid;
     float pos = 0.0f, neg = 0.0f;
@@ -306,14 +313,16 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
       if (wj > 0.0f) pos = fmaf(wj, bf16_to_f32(qf[j][e]), pos);
       else if (wj < 0.0f) neg = fmaf(-wj, bf16_to_f32(qf[j][e]), neg);
     }
-    const uint16_t bp = f32_to_bf16(pos), bn = f32_to_bf16(neg);
+    float lin = 0.5f * pos;
+    for (int a = 0; a < R; ++a) lin = fmaf(0.5f * wrow[sel[a]], bf16_to_f32(qf[sel[a]][e]), lin);
+    const uint16_t bl = f32_to_bf16(lin), bn = f32_to_bf16(neg);
     uint16_t* prow = p.plan_q + static_cast<size_t>(t) * kPlanRows * kD;
-    prow[kRetained * kD + e] = bp;
+    prow[kRetained * kD + e] = bl;
     prow[(kRetained + 1) * kD + e] = bn;
     for (int a = 0; a < R; ++a) prow[a * kD + e] = qrow[sel[a] * kD + e];
-    const float dp = pos - bf16_to_f32(bp), dn = neg - bf16_to_f32(bn);
-    // reduce: ||pos||^2, ||neg||^2, ||dp||^2, ||dn||^2
-    float v[4] = {pos * pos, neg * neg, dp * dp, dn * dn};
+    const float dl = lin - bf16_to_f32(bl), dn = neg - bf16_to_f32(bn);
+    // reduce: ||pos||^2, ||neg||^2, ||dl||^2, ||dn||^2
+    float v[4] = {pos * pos, neg * neg, dl * dl, dn * dn};
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = warp_sum(v[i]);
     __shared__ float r4[4][4];
@@ -334,10 +343,12 @@ __global__ void __launch_bounds__(128) plan_kernel(const PlanParams p) {
       }
       float* ps = p.plan_s + static_cast<size_t>(t) * kPlanScalars;
       for (int a = 0; a < R; ++a) {
-        ps[a] = wrow[sel[a]];
-        ps[kRetained + a] = 0.5f * alpha[a];
+        ps[a] = 0.5f * wrow[sel[a]] + 0.5f * alpha[a];  // coefficient of |d_a|
+        ps[kRetained + a] = 0.0f;
       }
-      const float C = 0.5f * beta + 0.5f * n[2] + n[3] + S * (1.0f / 1024.0f);
+      // C: the residual term, the bf16 rounding of L and q_neg, and 2^-10 S
+      // for the fp32 arithmetic (S bounds every product the bound sums)
+      const float C = 0.5f * beta + n[2] + n[3] + S * (1.0f / 1024.0f);
       ps[28] = C * (1.0f + 1.0f / 1024.0f);
       ps[29] = p.tau[t];
       ps[30] = 0.0f;
@@ -371,7 +382,6 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
   }
   if (tid == 0) {
     p.row_flags[t] = kRowRefined;
-    p.refine_len[t] = count;
     s_base = 0;
   }
   __syncthreads();
@@ -379,9 +389,16 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
   const int64_t words = pos / 32 + 1;
   const uint32_t* bm = p.bitmask + static_cast<size_t>(t) * p.mask_words;
   int32_t* ids = p.surv_ids + static_cast<size_t>(t) * p.cap_row;
+  // keys of the row's group's shared stream (in the words of the group's
+  // common range) are refined there, not here
+  const int g = t >> 2;
+  const uint32_t* gm = (p.group_mask && p.group_len[g] > 0) ? p.group_mask + static_cast<size_t>(g) * p.mask_words
+                                                            : nullptr;
+  const int64_t gwords = (p.q_offset + 4 * static_cast<int64_t>(g)) / 32 + 1;
   for (int64_t base = 0; base < words; base += 256) {
     const int64_t wi = base + tid;
     uint32_t word = wi < words ? bm[wi] : 0u;
+    if (gm && wi < gwords) word &= ~gm[wi];
     if (wi == words - 1 && (pos & 31) != 31) word &= (2u << (pos & 31)) - 1u;  // keys beyond pos
     const int c = __popc(word);
     int incl = c;
@@ -405,6 +422,70 @@ __global__ void __launch_bounds__(256) compact_kernel(const CompactParams p) {
     if (tid == 255) s_base = before + incl;
     __syncthreads();
   }
+  if (tid == 0) p.refine_len[t] = min(s_base, p.cap_row);  // the row's own list
+}
+
+// ---------------------------------------------------------------------------
+// Shared refine stream of one group of four consecutive rows (one CTA of 256
+// threads per group; "DoSA" notes, annotation WFZZA9CL, step 3).  Only full
+// groups whose four rows keep their survivor lists take part.  A key in the
+// group's common range (keys 0 .. position of the group's first row) kept by
+// at least two of the rows goes to the group's list: it is gathered once and
+// scored exactly for all four rows; each row's own list leaves it out.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) share_kernel(const ShareParams p) {
+  __shared__ int s_scan[256 / 32];
+  __shared__ int s_base;
+  if (p.skip && *p.skip) return;
+  const int g = blockIdx.x;
+  const int64_t t0 = 4 * static_cast<int64_t>(g);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  bool share = t0 + 4 <= p.T_q && (*p.err & kErrSeed) == 0;
+  for (int r = 0; r < 4 && share; ++r) share = p.surv_count[t0 + r] <= p.cap_row;
+  if (!share) {
+    if (tid == 0) p.group_len[g] = 0;
+    return;
+  }
+  if (tid == 0) s_base = 0;
+  __syncthreads();
+  const int64_t pos = p.q_offset + t0;  // the group's first row sees keys 0..pos
+  const int64_t words = pos / 32 + 1;
+  const uint32_t* bm = p.bitmask + static_cast<size_t>(t0) * p.mask_words;
+  uint32_t* gm = p.group_mask + static_cast<size_t>(g) * p.mask_words;
+  int32_t* ids = p.group_ids + static_cast<size_t>(g) * p.cap_row;
+  for (int64_t base = 0; base < words; base += 256) {
+    const int64_t wi = base + tid;
+    uint32_t word = 0u;
+    if (wi < words) {
+      const uint32_t a = bm[wi], b = bm[p.mask_words + wi], c = bm[2 * p.mask_words + wi],
+                     d = bm[3 * p.mask_words + wi];
+      word = (a & b) | (a & c) | (a & d) | (b & c) | (b & d) | (c & d);  // at least two of four
+      if (wi == words - 1 && (pos & 31) != 31) word &= (2u << (pos & 31)) - 1u;
+      gm[wi] = word;
+    }
+    const int cnt = __popc(word);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_scan[wid] = incl;
+    __syncthreads();
+    int before = s_base;
+    for (int w2 = 0; w2 < wid; ++w2) before += s_scan[w2];
+    int at = before + incl - cnt;
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (at < p.cap_row) ids[at] = static_cast<int32_t>(wi * 32 + bit);
+      ++at;
+    }
+    __syncthreads();
+    if (tid == 255) s_base = before + incl;
+    __syncthreads();
+  }
+  if (tid == 0) p.group_len[g] = min(s_base, p.cap_row);
 }
 
 // ---------------------------------------------------------------------------
@@ -471,10 +552,11 @@ __global__ void __launch_bounds__(256) decide_kernel(const DecideParams p) {
   }
 }
 
-// Sums for dsa_stats (one CTA): out[0] survivor pairs, [1] refined pairs,
-// [2] rows recovered after screening, [3] bypassed rows, [4] screened pairs,
-// [5] records the final selection read (seed Top-k + refined candidates of
-// the rows it finished).
+// Sums for dsa_stats (one CTA): out[0] survivor pairs, [1] refined pairs
+// (exact scores computed: own lists, plus four per shared key), [2] rows
+// recovered after screening, [3] bypassed rows, [4] screened pairs, [5]
+// records the final selection read (seed Top-k + refined candidates of the
+// rows it finished), [6] shared keys.
 __global__ void __launch_bounds__(256) stats_kernel(const StatsParams p) {
   unsigned long long a = 0, b = 0, c = 0, by = 0, sc = 0, rec = 0;
   for (int64_t t = threadIdx.x; t < p.T_q; t += blockDim.x) {
@@ -491,19 +573,33 @@ __global__ void __launch_bounds__(256) stats_kernel(const StatsParams p) {
       continue;
     }
     rec += static_cast<unsigned long long>(p.topk);
+    auto unit_recs = [&](const int32_t* m) {
+      unsigned long long r = static_cast<unsigned long long>(min(max(m[1], 0), p.lay.keep_cap));
+      for (int q = 0; q < 4; ++q) r += static_cast<unsigned long long>(min(max(m[2 + q], 0), p.lay.app_cap));
+      return r;
+    };
     const int u0 = p.seq_ubeg[t], nu = p.seq_ucnt[t];
-    for (int u = u0; u < u0 + nu; ++u) {
-      const int32_t* m = p.meta + static_cast<size_t>(u) * kMetaInts;
-      rec += static_cast<unsigned long long>(min(max(m[1], 0), p.lay.keep_cap));
-      for (int r = 0; r < 4; ++r) rec += static_cast<unsigned long long>(min(max(m[2 + r], 0), p.lay.app_cap));
+    for (int u = u0; u < u0 + nu; ++u) rec += unit_recs(p.meta + static_cast<size_t>(u) * kMetaInts);
+    if (p.group_len) {
+      const int64_t g = t >> 2;
+      const int g0 = p.gs_ubeg[g], gn = p.gs_ucnt[g];
+      for (int u = g0; u < g0 + gn; ++u) rec += unit_recs(p.meta2 + (static_cast<size_t>(u) * 4 + (t & 3)) * kMetaInts);
     }
   }
+  unsigned long long shared = 0;
+  if (p.group_len)
+    for (int64_t g = threadIdx.x; g < (p.T_q + 3) / 4; g += blockDim.x) {
+      const unsigned long long n = static_cast<unsigned long long>(p.group_len[g]);
+      shared += n;
+      b += 4 * n;
+    }
   atomicAdd(&p.out[0], a);
   atomicAdd(&p.out[1], b);
   atomicAdd(&p.out[2], c);
   atomicAdd(&p.out[3], by);
   atomicAdd(&p.out[4], sc);
   atomicAdd(&p.out[5], rec);
+  atomicAdd(&p.out[6], shared);
 }
 
 cudaError_t launch_seed_prep(const SeedPrepParams& p, cudaStream_t st) {
@@ -524,6 +620,12 @@ cudaError_t launch_plan(int H, const PlanParams& p, cudaStream_t st) {
   if (H == 64) plan_kernel<64><<<static_cast<unsigned>(p.T_q), 128, 0, st>>>(p);
   else if (H == 32) plan_kernel<32><<<static_cast<unsigned>(p.T_q), 128, 0, st>>>(p);
   else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_share(const ShareParams& p, cudaStream_t st) {
+  const int64_t groups = (p.T_q + 3) / 4;
+  if (groups > 0) share_kernel<<<static_cast<unsigned>(groups), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -99,6 +99,7 @@ enum ScoreMode : int {
   kModeDecode = 1,   // one query per sequence; keys 0..seq_len[b]-1 of its own cache
   kModeGathered = 2, // query groups; keys are a gathered list (all visible), ids remapped
   kModeRefine = 3,   // one query row per unit (table like decode); keys gathered by id
+  kModeRefineShared = 4,  // G consecutive rows per unit (table over row groups); keys gathered by id
 };
 
 // Epilogue variants of the fused kernel.
@@ -145,6 +146,12 @@ struct ScoreParams {
   // key [T_k] (the bf16 kernels ignore them)
   const float* q_scale;
   const float* k_scale;
+  // paged decode: sequence b's key i sits at row block_table[b][i / page_size]
+  // * page_size + i % page_size of the page pool (null: contiguous caches)
+  const int32_t* block_table;
+  int max_blocks;
+  int page_size;    // a multiple of 64
+  int64_t n_pages;
   // refine: survivor key ids per row (stride surv_stride), the key matrix they
   // index, and an initial admission threshold record per row
   const int32_t* surv_ids;
@@ -172,6 +179,14 @@ struct SelectParams {
   const int32_t* meta;
   const int32_t* seq_ubeg;  // decode / refine
   const int32_t* seq_ucnt;  // decode / refine
+  // optional second candidate source (the DoSA shared refine stream): units
+  // of G2 consecutive rows; row r reads units ubeg2[r / G2] .. + ucnt2[r / G2]
+  // as query r % G2
+  const uint64_t* cand2;
+  const int32_t* meta2;
+  const int32_t* ubeg2;
+  const int32_t* ucnt2;
+  int G2;
   const uint64_t* extra_rec;  // optional [n_rows][rec_stride] extra records (0 = none) merged per row
   int rec_stride;             // row stride of extra_rec / out_rec (>= topk, even)
   const int32_t* row_flags;   // optional: only rows with a non-zero flag are written
@@ -241,6 +256,8 @@ cudaError_t launch_score(int H, int G, int eg, const CUtensorMap& tmap_q, const 
 // The same fused kernel on FP8 (E4M3) query and key tiles (prefill only).
 cudaError_t launch_score_fp8(int H, int G, int eg, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                              const ScoreParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_refine_shared(int H, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k, const ScoreParams& p,
+                                 int grid, cudaStream_t stream);
 cudaError_t launch_screen(const CUtensorMap& tmap_plan, const CUtensorMap& tmap_k, const ScoreParams& p,
                           int grid, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);

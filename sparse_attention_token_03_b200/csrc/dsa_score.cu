@@ -210,12 +210,18 @@ struct Unit {
 template <int G>
 __device__ __forceinline__ Unit unit_geometry(const ScoreParams& p, int u, int H) {
   Unit U;
-  if (p.mode == kModeDecode || p.mode == kModeRefine) {
+  if (p.mode == kModeDecode || p.mode == kModeRefine || p.mode == kModeRefineShared) {
+    // b: the sequence / row, or (shared refine) the group of G rows
     const int b = p.unit_tab[3 * u + 0];
     U.slot = u;
-    U.row0 = b;
-    U.rows = 1;
-    U.q_row = static_cast<int64_t>(b) * H;
+    if (p.mode == kModeRefineShared) {
+      U.row0 = static_cast<int64_t>(b) * G;
+      U.rows = static_cast<int>(p.T_q - U.row0 < G ? p.T_q - U.row0 : G);
+    } else {
+      U.row0 = b;
+      U.rows = 1;
+    }
+    U.q_row = U.row0 * H;
     U.k_row = (p.mode == kModeDecode) ? static_cast<int64_t>(b) * p.t_cap : 0;
     U.tile_lo = p.unit_tab[3 * u + 1];
     U.tile_hi = p.unit_tab[3 * u + 2];
@@ -248,8 +254,16 @@ __device__ __forceinline__ Unit unit_geometry(const ScoreParams& p, int u, int H
   return U;
 }
 
+__device__ __forceinline__ bool gathered_ids(const ScoreParams& p) {
+  return p.mode == kModeRefine || p.mode == kModeRefineShared;
+}
 __device__ __forceinline__ bool tabled(const ScoreParams& p) {
-  return p.mode == kModeDecode || p.mode == kModeRefine;
+  return p.mode == kModeDecode || gathered_ids(p);
+}
+// Row of the key-id table a refine unit reads (its row, or its row group).
+template <int G>
+__device__ __forceinline__ int64_t id_row(const ScoreParams& p, const Unit& U) {
+  return p.mode == kModeRefineShared ? U.row0 / G : U.row0;
 }
 __device__ __forceinline__ int cta_unit_begin(const ScoreParams& p) {
   return tabled(p) ? p.cta_ubeg[blockIdx.x] : static_cast<int>(blockIdx.x);
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     mbar_init(bar_q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       // gathered key tiles are signalled by all 32 producer lanes, TMA tiles by one
-      mbar_init(bar_k_full(s), p.mode == kModeRefine ? 32 : 1);
+      mbar_init(bar_k_full(s), gathered_ids(p) ? 32 : 1);
       mbar_init(bar_k_empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -342,7 +356,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
   if (warp < score_epi_warp0(EG)) {
    // one setmaxnreg for the whole control warpgroup
    if constexpr (EG >= 2) regs_dec<regs_ctl(EG)>();
-   if (!F8 && warp == 0 && p.mode == kModeRefine && !p.stall_loads) {
+   if (!F8 && warp == 0 && gathered_ids(p) && !p.stall_loads) {
     // ------------------------------------------------ producer (gathered keys)
     // Survivor keys are gathered row by row with 16-byte cp.async into the
     // 128B-swizzled layout the MMA reads.  A stage is signalled LAG tiles
@@ -375,7 +389,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       ++qi;
-      const int32_t* ids = p.surv_ids + U.row0 * p.surv_stride;
+      const int32_t* ids = p.surv_ids + id_row<G>(p, U) * p.surv_stride;
       const int64_t n = U.vis_base;
       for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
         const int s = kt % NS;
@@ -420,15 +434,50 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         if (u + u_step < u_end) {  // warm L2 with the next unit's query tile
           const Unit V = unit_geometry<G>(p, u + u_step, H);
           tma_prefetch_l2_2d(&tmap_q, 0, static_cast<int32_t>(V.q_row));
-          tma_prefetch_l2_2d(&tmap_q, 64, static_cast<int32_t>(V.q_row));
+          if constexpr (!F8) tma_prefetch_l2_2d(&tmap_q, 64, static_cast<int32_t>(V.q_row));
         }
+        // paged key cache: each 64-key half of a tile lies in one page (page
+        // sizes are multiples of 64); the block-table entries of tile t + 1
+        // are read while tile t's stage is awaited.  Keys past the sequence's
+        // length read page 0 and are masked by the epilogue.
+        int32_t pg[2] = {0, 0}, pn[2] = {0, 0};
+        auto lookup = [&](int64_t t, int32_t (&o)[2]) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int64_t key0 = t * kTileKeys + 64 * h;
+            o[h] = key0 < U.vis_base ? p.block_table[U.row0 * p.max_blocks + key0 / p.page_size] : 0;
+          }
+        };
+        if (!F8 && p.block_table) lookup(U.tile_lo, pg);
         for (int64_t t = U.tile_lo; t < U.tile_hi; ++t) {
           const int s = kt % NS;
+          if (!F8 && p.block_table && t + 1 < U.tile_hi) lookup(t + 1, pn);
           if (!(ok = mbar_wait(bar_k_empty(s), ((kt / NS) & 1) ^ 1, s_abort, p.err, wlim))) break;
           mbar_arrive_expect_tx(bar_k_full(s), L.k_stage());
-          const int32_t krow = static_cast<int32_t>(U.k_row + t * kTileKeys);
-          tma_load_2d(sK + s * L.k_stage(), &tmap_k, 0, krow, bar_k_full(s));
-          if constexpr (!F8) tma_load_2d(sK + s * L.k_stage() + L.k_sub(), &tmap_k, 64, krow, bar_k_full(s));
+          if (!F8 && p.block_table) {
+            // pages of a multiple of 128 keys hold whole tiles: one box of 128
+            // rows per column half (the key map's box is 128 rows then);
+            // 64-key pages take one box of 64 rows per half tile
+            const int nh = (p.page_size % kTileKeys == 0) ? 1 : 2;
+            for (int h = 0; h < nh; ++h) {
+              const int64_t key0 = t * kTileKeys + 64 * h;
+              int32_t page = pg[h];
+              if (page < 0 || page >= p.n_pages) {
+                atomicOr(p.err, kErrOverflow);
+                page = 0;
+              }
+              const int32_t prow = static_cast<int32_t>(static_cast<int64_t>(page) * p.page_size + key0 % p.page_size);
+              const uint32_t half = static_cast<uint32_t>(h) * 64u * 128u;
+              tma_load_2d(sK + s * L.k_stage() + half, &tmap_k, 0, prow, bar_k_full(s));
+              tma_load_2d(sK + s * L.k_stage() + L.k_sub() + half, &tmap_k, 64, prow, bar_k_full(s));
+            }
+            pg[0] = pn[0];
+            pg[1] = pn[1];
+          } else {
+            const int32_t krow = static_cast<int32_t>(U.k_row + t * kTileKeys);
+            tma_load_2d(sK + s * L.k_stage(), &tmap_k, 0, krow, bar_k_full(s));
+            if constexpr (!F8) tma_load_2d(sK + s * L.k_stage() + L.k_sub(), &tmap_k, 64, krow, bar_k_full(s));
+          }
           ++kt;
         }
       }
@@ -497,11 +546,13 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     // d_neg; C carries the residual, bf16-rounding and fp32 slack terms).  A
     // visible non-seed key survives unless U < tau ("DoSA", step 2: prune only
     // when the bound is strictly below the threshold, keep when unsure).
-    // Each retained head's term is evaluated as (w_i/2) d_i + (w_i/2 + alpha_i/2)
-    // |d_i| (equal in exact arithmetic; two FMAs, the second with an
-    // absolute-value operand); the fp32 rounding of the coefficients and of
-    // the sum lies far inside the 2^-10 S ||k|| part of C.  The coefficients
-    // of this thread's queries stay in registers for the whole unit.
+    // Since w max(d, 0) = (w d + w |d|) / 2, the linear parts of every term
+    // are one plan row L (its dot d_L comes from the MMA) and the rest is
+    // U = d_L + sum_i c_i |d_i| - max(d_neg, 0) + C ||k||, one FMA with an
+    // absolute-value operand per retained head; the fp32 rounding of the
+    // coefficients and of the sum lies far inside the 2^-10 S ||k|| part of
+    // C.  The coefficients of this thread's queries stay in registers for the
+    // whole unit.
     if constexpr (EG >= 2) regs_inc<regs_epi(EG)>();
     const int e = (warp - score_epi_warp0(EG)) >> 2;
     const int quarter = warp & 3;
@@ -511,18 +562,14 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
     bool ok = true;
     for (int u = u_begin; ok && u < u_end; u += u_step) {
       const Unit U = unit_geometry<G>(p, u, H);
-      float c1[GQ][kRetained], c2[GQ][kRetained], cc[GQ], tau[GQ];
+      float c2[GQ][kRetained], cc[GQ], tau[GQ];
 #pragma unroll
       for (int i = 0; i < GQ; ++i) {
         const int qq = q_lo + i;
         const bool on = qq < U.rows;
         const float* ps = p.plan_s + (U.row0 + (on ? qq : 0)) * kPlanScalars;
 #pragma unroll
-        for (int r = 0; r < kRetained; ++r) {
-          const float w = on ? __ldg(ps + r) : 0.0f, ah = on ? __ldg(ps + kRetained + r) : 0.0f;
-          c1[i][r] = 0.5f * w;
-          c2[i][r] = 0.5f * w + ah;
-        }
+        for (int r = 0; r < kRetained; ++r) c2[i][r] = on ? __ldg(ps + r) : 0.0f;
         cc[i] = on ? __ldg(ps + 28) : 0.0f;
         tau[i] = on ? __ldg(ps + 29) : 0.0f;
       }
@@ -546,14 +593,15 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         for (int i = 0; i < GQ; ++i) {
           if (i + 1 < GQ) tmem_ld16(trow + (i + 1) * H, xb[(i + 1) & 1]);
           const uint32_t* d = xb[i & 1];
-          float ub = 0.0f;
+          // two chains over the retained heads, then the linear row, the
+          // negative fold and the slack
+          float u0 = __uint_as_float(d[kRetained]), u1 = 0.0f;
 #pragma unroll
-          for (int r = 0; r < kRetained; ++r) {
-            const float x = __uint_as_float(d[r]);
-            ub = fmaf(c1[i][r], x, ub);
-            ub = fmaf(c2[i][r], fabsf(x), ub);
+          for (int r = 0; r < kRetained; r += 2) {
+            u0 = fmaf(c2[i][r], fabsf(__uint_as_float(d[r])), u0);
+            u1 = fmaf(c2[i][r + 1], fabsf(__uint_as_float(d[r + 1])), u1);
           }
-          ub = fmaf(0.5f, __uint_as_float(d[kRetained]), ub);
+          float ub = u0 + u1;
           ub -= fmaxf(__uint_as_float(d[kRetained + 1]), 0.0f);
           ub = fmaf(cc[i], kn, ub);
           const int qq = q_lo + i;
@@ -666,8 +714,8 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         const int64_t key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
-        if (p.mode == kModeRefine && key_local < U.vis_base)
-          key_id = static_cast<uint32_t>(p.surv_ids[U.row0 * p.surv_stride + key_local]);
+        if (gathered_ids(p) && key_local < U.vis_base)
+          key_id = static_cast<uint32_t>(p.surv_ids[id_row<G>(p, U) * p.surv_stride + key_local]);
         // this warpgroup's GQ x H dot products, read in 16-column chunks: the
         // next chunk's TMEM load overlaps the current chunk's head sums
         constexpr int CPQ = H / 16, NC = GQ * CPQ;
@@ -933,6 +981,18 @@ cudaError_t launch_score_fp8(int H, int G, int eg, const CUtensorMap& tq, const 
   if (H == 64 && G == 4 && eg == 2) return launch_score_t<64, 4, 8, 2, kEpiScore, true>(tq, tk, p, grid, stream);
   if (H == 32 && G == 8 && eg == 4) return launch_score_t<32, 8, 6, 4, kEpiScore, true>(tq, tk, p, grid, stream);
   if (H == 32 && G == 8 && eg == 2) return launch_score_t<32, 8, 6, 2, kEpiScore, true>(tq, tk, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+// The DoSA shared refine stream: four consecutive rows per unit (N = 4 H),
+// survivor keys gathered by id.
+cudaError_t launch_refine_shared(int H, const CUtensorMap& tq, const CUtensorMap& tk, const ScoreParams& p0,
+                                 int grid, cudaStream_t stream) {
+  ScoreParams p = p0;
+  take_wait_injection(p);
+  if (p.mode != kModeRefineShared) return cudaErrorInvalidValue;
+  if (H == 64) return launch_score_t<64, 4, 4, 4>(tq, tk, p, grid, stream);
+  if (H == 32) return launch_score_t<32, 4, 5, 2>(tq, tk, p, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -189,25 +189,37 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
   const int G = (p.mode == kModeDecode) ? 1 : p.G;
   const CandLayout lay = p.lay;
 
-  // segment sg = 5 * unit + region of the row's candidate buffers; one more
-  // segment holds the row's extra records when given
+  // segment sg = 5 * unit + region of the row's candidate buffers (its own
+  // units, then the units of the second source); one more segment holds the
+  // row's extra records when given
+  int n_u2 = 0, slot2 = 0, q2 = 0;
+  if (p.cand2) {
+    const int64_t g2 = row / p.G2;
+    slot2 = p.ubeg2[g2];
+    n_u2 = p.ucnt2[g2];
+    q2 = static_cast<int>(row % p.G2);
+  }
+  const int n_own = 5 * R.n_u;
   auto unit_meta = [&](int u) -> const int32_t* {
+    if (u >= R.n_u) return p.meta2 + (static_cast<size_t>(slot2 + u - R.n_u) * p.G2 + q2) * kMetaInts;
     return p.meta + (static_cast<size_t>(R.slot_lo + u) * G + R.q) * kMetaInts;
   };
   auto segment = [&](int sg, int& cnt) -> const uint64_t* {
-    if (sg == 5 * R.n_u) {
+    if (sg == 5 * (R.n_u + n_u2)) {
       cnt = p.topk;
       return p.extra_rec + static_cast<size_t>(row) * p.rec_stride;
     }
     const int u = sg / 5, r = sg % 5;
-    const size_t qi = static_cast<size_t>(R.slot_lo + u) * G + R.q;
-    const int32_t* mt = p.meta + qi * kMetaInts;
+    const bool second = sg >= n_own;
+    const size_t qi = second ? static_cast<size_t>(slot2 + u - R.n_u) * p.G2 + q2
+                             : static_cast<size_t>(R.slot_lo + u) * G + R.q;
+    const int32_t* mt = (second ? p.meta2 : p.meta) + qi * kMetaInts;
     const int cap = (r == 0) ? lay.keep_cap : lay.app_cap;
     cnt = min(max(mt[1 + r], 0), cap);  // counts are always in range; clamp defensively
-    return p.cand + qi * lay.query_recs() + static_cast<size_t>(mt[0] & 1) * lay.half_recs() +
+    return (second ? p.cand2 : p.cand) + qi * lay.query_recs() + static_cast<size_t>(mt[0] & 1) * lay.half_recs() +
            lay.region_off(r);
   };
-  const int n_seg = 5 * R.n_u + (p.extra_rec ? 1 : 0);
+  const int n_seg = 5 * (R.n_u + n_u2) + (p.extra_rec ? 1 : 0);
   const bool table = n_seg <= kSelSegs;
 
   // 1. warp 0: segment table (offsets of a flattened index), total count and
@@ -222,7 +234,7 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
       const uint64_t* ptr = nullptr;
       if (sg < n_seg) {
         ptr = segment(sg, c);
-        if (sg == 5 * R.n_u) {
+        if (sg == 5 * (R.n_u + n_u2)) {
           const uint64_t kth = ptr[p.topk - 1];
           thr = kth > thr ? kth : thr;
         } else if (sg % 5 == 0) {

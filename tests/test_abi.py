@@ -94,3 +94,22 @@ def test_binding_has_the_header_names():
     missing = sorted(n for n in names - {"dsa_last_error_string"} if not callable(getattr(dsa, n, None)))
     assert not missing, missing
     assert set(dsa.__all__) >= names - {"dsa_last_error_string"}
+
+
+def test_history_seeds_validation_without_gpu():
+    L = dsa.lib()
+    P = ctypes.c_void_p
+    dummy = P(256)
+    need = L.dsa_index_seeds_from_history_workspace_bytes(100_003)
+    # counts and a 65536-bin histogram at least; tile prefixes for 98 tiles
+    assert need >= 4 * 100_003 + 4 * 65536 and need % 256 == 0
+    assert L.dsa_index_seeds_from_history_workspace_bytes(0) == 0
+    # n_seed outside [1, n_keys], bad sizes, nulls, short or misaligned workspace
+    assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 11, dummy, dummy, need, None) == -1
+    assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 0, dummy, dummy, need, None) == -1
+    assert L.dsa_index_seeds_from_history(dummy, -1, 8, 10, 5, dummy, dummy, need, None) == -1
+    assert L.dsa_index_seeds_from_history(None, 4, 8, 10, 5, dummy, dummy, need, None) == -1
+    assert L.dsa_index_seeds_from_history(dummy, 1 << 30, 8, 10, 5, dummy, dummy, need, None) == -1
+    assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 5, dummy, P(264), need, None) == -1
+    small = L.dsa_index_seeds_from_history_workspace_bytes(10)
+    assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 5, dummy, dummy, small - 1, None) == -3

@@ -50,6 +50,20 @@ def run_both(x, topk, seeds, workspace=None):
     return di.cpu().numpy(), ds.cpu().numpy(), pi.cpu().numpy(), ps.cpu().numpy(), st
 
 
+def check_refine_counts(st, all_refined=False):
+    """refined_pairs counts the exact scores computed: one per survivor in a
+    row's own list, four per key of a group's shared stream (a shared key is
+    a survivor of at least two of the group's four rows)."""
+    shared = st["shared_keys"]
+    assert shared >= 0
+    if all_refined:  # no row recovered: every survivor was refined once
+        own = st["refined_pairs"] - 4 * shared
+        assert own >= 0 and st["survivor_pairs"] > 0
+        assert own + 2 * shared <= st["survivor_pairs"] <= own + 4 * shared
+    else:
+        assert st["refined_pairs"] - 4 * shared <= st["survivor_pairs"]
+
+
 def screened_rows(T_q, st):
     """Rows that went through the screen: all of them, or only the probe when
     the probe sent the rest of the chunk to the dense pass."""
@@ -79,7 +93,7 @@ def test_pruned_equals_dense_bitwise_and_oracle(recipe, H):
     T_q = T_k - off
     assert st["screened_pairs"] == expected_screened_pairs(off, T_q, len(seeds), st)
     assert 0 <= st["survivor_pairs"] <= st["screened_pairs"]
-    assert st["refined_pairs"] <= st["survivor_pairs"]
+    check_refine_counts(st)
     print(recipe, st)
 
 
@@ -110,8 +124,9 @@ def test_pruned_refine_path_with_a_tight_bound(H):
     print("tight bound", H, st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
     assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
     assert st["recovered_rows"] == 0
-    assert st["refined_pairs"] == st["survivor_pairs"] > 0
+    check_refine_counts(st, all_refined=True)
     assert st["survivor_pairs"] < 0.2 * st["screened_pairs"]
+    assert st["shared_keys"] > 0  # the rows repeat one query: their survivors are shared
     rows = np.array([0, 11, 23])
     oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
     check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, f"tight {H}")
@@ -287,7 +302,8 @@ def test_full_size_pruned_refine_path_without_recovery():
     print("full-size tight bound", st, "filter rate", 1 - st["survivor_pairs"] / st["screened_pairs"])
     assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
     assert st["bypassed_rows"] == 0 and st["recovered_rows"] == 0
-    assert st["refined_pairs"] == st["survivor_pairs"] > 0
+    check_refine_counts(st, all_refined=True)
+    assert st["shared_keys"] > 0
     assert st["screened_pairs"] == expected_screened_pairs(wl.q_offset, wl.T_q, wl.n_seed, st)
     rows = np.array([0, 4095, wl.T_q - 1])
     oi, osc, amax, score_of = oracle_prefill_rows(x, rows, wl.topk)
@@ -310,3 +326,35 @@ def test_probe_sends_an_unfilterable_chunk_to_the_dense_pass():
     rows = np.array([0, 127, 128, 700, T_q - 1])
     oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
     check_rows(pi[rows], ps[rows], oi, osc, amax, off + rows + 1, topk, score_of, "bypass")
+
+
+def test_shared_refine_stream_mixes_shared_and_own_keys():
+    # groups of four rows whose queries differ: the shared stream holds only
+    # the keys two or more rows keep; the result is still the dense one bit
+    # for bit.  Rows 0-3 repeat query A, rows 4-7 alternate A and B, rows
+    # 8-11 are four different queries built like A
+    T_q, off, topk = 12, 6000, 128
+    x, _ = _tight_bound_chunk("causal_16k_h64", T_q, off + T_q, off, topk, 409, 300)
+    rng = np.random.default_rng(3)
+    qb = x["q"][0].copy()
+    qb[:14] = np.flip(qb[:14], axis=1)  # another query with the same head structure
+    x["q"][5] = qb
+    x["q"][7] = qb
+    for t in range(8, 12):
+        qt = x["q"][0].copy()
+        qt[:14] = qt[:14][rng.permutation(14)][:, rng.permutation(128)]
+        x["q"][t] = qt
+    # seeds: every distinct query's Top-k among the keys before the chunk
+    # (a tight threshold for every row), plus random keys
+    top = [oracle.prefill_topk(x["q"][t:t + 1], x["w"][t:t + 1], x["k"][:off], off - 1, topk)[0][0]
+           for t in (0, 5, 8, 9, 10, 11)]
+    top = np.unique(np.concatenate(top))
+    seeds = np.concatenate([top, random_distinct_keys(14, 0, off, 300, exclude=top)]).astype(np.int32)
+    di, ds, pi, ps, st = run_both(x, topk, seeds)
+    print("mixed groups", st)
+    assert np.array_equal(pi, di) and np.array_equal(ps.view(np.uint32), ds.view(np.uint32))
+    assert st["recovered_rows"] == 0
+    check_refine_counts(st, all_refined=True)
+    rows = np.arange(T_q)
+    oi, osc, amax, score_of = oracle_prefill_rows(x, rows, topk)
+    check_rows(pi, ps, oi, osc, amax, off + rows + 1, topk, score_of, "mixed groups")
