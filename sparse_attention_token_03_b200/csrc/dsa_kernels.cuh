@@ -75,6 +75,7 @@ static_assert(hist_bin(hist_edge(1)) == 1 && hist_bin(hist_edge(1) - 1) == 0 &&
 // The epilogue publishes append counts and checks for overflow every
 // kCheckTiles tiles; a warp appends at most 32 records per query per tile.
 constexpr int kCheckTiles = 16;
+static_assert((kCheckTiles & (kCheckTiles - 1)) == 0, "the check cadence is a power of two");
 
 struct CandLayout {
   int keep_cap;  // records kept by a compaction (>= topk), multiple of 32

@@ -284,15 +284,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 // +0, and w / 2 is exact for normal weights, so the product is the same real
 // number and the FMA rounds once either way.  The add (with an absolute-value
 // operand) and the FMA run on the FMA pipe, where a max would take the ALU,
-// and chains c and c+1 advance together in one paired FMA (__ffma2_rn, per
-// component the same operation as fmaf).  head_acc16 adds 16 consecutive
+// and heads j and j+1 (chains c and c+1) advance together in one paired add
+// and one paired FMA (__fadd2_rn, __ffma2_rn: per component the same
+// operations as + and fmaf).  head_acc16 adds 16 consecutive
 // heads (j0 .. j0+15, j0 a multiple of 16) to the chains, held as pairs
 // a[c/2] = (a_c, a_c+1); wh holds the HALVED weights of those heads.
 __device__ __forceinline__ void head_acc16(float2 (&a)[4], const uint32_t (&x)[16], const float* wh) {
 #pragma unroll
   for (int j = 0; j < 16; j += 2) {
     const float x0 = __uint_as_float(x[j]), x1 = __uint_as_float(x[j + 1]);
-    a[(j & 7) >> 1] = __ffma2_rn(make_float2(wh[j], wh[j + 1]), make_float2(x0 + fabsf(x0), x1 + fabsf(x1)),
+    a[(j & 7) >> 1] = __ffma2_rn(make_float2(wh[j], wh[j + 1]),
+                                 __fadd2_rn(make_float2(x0, x1), make_float2(fabsf(x0), fabsf(x1))),
                                  a[(j & 7) >> 1]);
   }
 }

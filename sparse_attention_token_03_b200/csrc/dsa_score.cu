@@ -667,6 +667,17 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       epi_sync(bar);
       // with one or two warpgroups, the halved head weights stay in registers
       // for the whole unit
+      // with four warpgroups the first 16 weights of the warpgroup's first
+      // query stay in registers too: a quarter (H = 64) or an eighth (H = 32)
+      // fewer shared-memory broadcasts per tile
+      constexpr int kWReg = kWSmem ? 16 : 0;
+      float wq[kWReg > 0 ? kWReg : 1];
+      if constexpr (kWReg > 0) {
+        const bool on = q_lo < U.rows;
+        const int64_t wrow0 = (U.row0 + (on ? q_lo : 0)) * H;
+#pragma unroll
+        for (int j = 0; j < kWReg; ++j) wq[j] = on ? half_weight(head_weight<F8>(p, wrow0 + j)) : 0.0f;
+      }
       float wr[kWSmem ? 1 : GQ][kWSmem ? 1 : H];
       if constexpr (!kWSmem) {
 #pragma unroll
@@ -707,11 +718,20 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
       };
       reload();
       bool nonfinite = false;  // a visible pair scored inf or NaN (reported at the unit's end)
-      for (int64_t t = U.tile_lo; ok && t < U.tile_hi; ++t) {
+      // per query: local keys below visq are visible (none for missing rows).
+      // Keys, tiles and these bounds fit 32 bits (T_k < 2^31).
+      int visq[GQ];
+#pragma unroll
+      for (int i = 0; i < GQ; ++i)
+        visq[i] = (q_lo + i < U.rows)
+                      ? static_cast<int>(p.mode == kModePrefill ? U.vis_base + q_lo + i : U.vis_base)
+                      : 0;
+      const int t_lo = static_cast<int>(U.tile_lo), t_hi = static_cast<int>(U.tile_hi);
+      for (int t = t_lo; ok && t < t_hi; ++t) {
         const int a = at & 1;
         if (!(ok = mbar_wait(bar_acc_full(a), (at >> 1) & 1, s_abort, p.err, wlim))) break;
         tc_fence_after();
-        const int64_t key_local = t * kTileKeys + row_in_tile;
+        const int key_local = t * kTileKeys + row_in_tile;
         uint32_t key_id = static_cast<uint32_t>(key_local);
         if (p.mode == kModeGathered && key_local < p.T_k) key_id = static_cast<uint32_t>(p.key_ids[key_local]);
         if (gathered_ids(p) && key_local < U.vis_base)
@@ -721,29 +741,34 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         constexpr int CPQ = H / 16, NC = GQ * CPQ;
         const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                               static_cast<uint32_t>(a * ACC_COLS + q_lo * H);
-        uint32_t xb[3][16];
+        // loads run RING - 1 chunks ahead of the math (one ahead in the
+        // one-query four-warpgroup epilogue, whose registers are tightest)
+        constexpr int RING = (kWSmem && GQ == 1) ? 2 : 3;
+        uint32_t xb[RING][16];
         float score[GQ];
         float2 acc[4];
-        tmem_ld16(trow, xb[0]);
-        if (NC > 1) tmem_ld16(trow + 16, xb[1]);
+#pragma unroll
+        for (int r = 0; r < RING - 1 && r < NC; ++r) tmem_ld16(trow + r * 16, xb[r]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-          // loads run two chunks ahead of the math
-          if (c + 2 < NC) tmem_ld16(trow + (c + 2) * 16, xb[(c + 2) % 3]);
+          if (c + RING - 1 < NC) tmem_ld16(trow + (c + RING - 1) * 16, xb[(c + RING - 1) % RING]);
           if (c % CPQ == 0) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.0f, 0.0f);
           }
           if constexpr (kWSmem) {
-            head_acc16_smem(acc, xb[c % 3], s_w + (q_lo + c / CPQ) * H + (c % CPQ) * 16);
+            if (c * 16 < kWReg)
+              head_acc16(acc, xb[c % RING], &wq[(c * 16) % (kWReg > 0 ? kWReg : 16)]);
+            else
+              head_acc16_smem(acc, xb[c % RING], s_w + (q_lo + c / CPQ) * H + (c % CPQ) * 16);
           } else {
-            head_acc16(acc, xb[c % 3], &wr[c / CPQ][(c % CPQ) * 16]);
+            head_acc16(acc, xb[c % RING], &wr[c / CPQ][(c % CPQ) * 16]);
           }
           if (c % CPQ == CPQ - 1) score[c / CPQ] = head_finish(acc);
-          if (c + 2 < NC) tmem_wait_ld();
+          if (c + RING - 1 < NC) tmem_wait_ld();
           // after the last load has landed, release the accumulator
-          if ((NC <= 2 && c == 0) || (NC > 2 && c + 3 == NC)) {
+          if (c == (NC > RING - 1 ? NC - RING : 0)) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_acc_empty(a));
@@ -760,12 +785,9 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
 #pragma unroll
         for (int i = 0; i < GQ; ++i) {
           const int qq = q_lo + i;
-          // keys of this tile visible to the query: local keys below lim
-          const int64_t lim64 = (p.mode == kModePrefill ? U.vis_base + qq : U.vis_base) - t * kTileKeys;
-          const int lim = lim64 < 0 ? 0 : (lim64 > kTileKeys ? kTileKeys : static_cast<int>(lim64));
           // one float compare rules out keys that cannot reach the threshold;
           // the exact record test runs only in warps where some lane passes
-          const bool vis = qq < U.rows && row_in_tile < lim;
+          const bool vis = key_local < visq[i];
           nonfinite = nonfinite || (vis && !(fabsf(score[i]) <= 3.402823466e38f));
           const bool pre = vis && score[i] >= thr_f[i];
           if (__any_sync(0xFFFFFFFFu, pre)) {
@@ -786,7 +808,7 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
         // publishes its append counts, raises each row's admission threshold
         // from the row's score-code histogram, and compacts buffers that
         // could overflow before the next check
-        if (((t - U.tile_lo) % kCheckTiles) != kCheckTiles - 1 && t + 1 != U.tile_hi) continue;
+        if (((t - t_lo) & (kCheckTiles - 1)) != kCheckTiles - 1 && t + 1 != t_hi) continue;
         if (lane == 0) {
 #pragma unroll
           for (int i = 0; i < GQ; ++i) s_wcnt[(q_lo + i) * 4 + quarter] = cnt[i];
