@@ -259,6 +259,40 @@ DSA_API int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_
                                                void* stream);
 
 /*
+ * Chunked prefill, dense and DoSA-pruned, over a paged key cache (the pages'
+ * port keeps keys in pages and reads them through page tables: "DoSA" notes,
+ * annotation LJZ23SXM).  Same computation, outputs and status bits as
+ * dsa_index_prefill / dsa_index_prefill_pruned on the keys
+ *     k(s) = k_pages[block_table[s / page_size]][s % page_size],  0 <= s < T_k.
+ * One bandwidth-bound pass first gathers those T_k keys into the workspace
+ * (2 x 256 bytes per key moved, against the O(T_q x T_k) scoring that
+ * follows); the scoring kernels then stream them as contiguous TMA tiles.
+ *   k_pages      device, [n_pages][page_size][128] bf16, 16-byte aligned;
+ *                page_size >= 1, n_pages * page_size < 2^31
+ *   block_table  device, [ceil(T_k / page_size)] int32 page ids of this
+ *                sequence; an id outside [0, n_pages) reads zeros and sets
+ *                status bit 1 (the pruned call with stats returns
+ *                DSA_EDEVICE for it)
+ *   workspace    256-byte aligned, of the *_paged_workspace_bytes() size:
+ *                the contiguous call's workspace (its status word at byte 0,
+ *                read with dsa_index_device_status; for the pruned call also
+ *                dsa_index_prefill_pruned_survivors), then the gathered keys.
+ *                The dense call accepts less and runs row blocks.
+ */
+DSA_API size_t dsa_index_prefill_paged_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk);
+DSA_API int dsa_index_prefill_paged(const uint16_t* q, const float* w, const uint16_t* k_pages, int64_t n_pages,
+                                    int page_size, const int32_t* block_table, int64_t q_offset, int64_t T_q,
+                                    int64_t T_k, int H, int d, int topk, int32_t* out_idx, float* out_score,
+                                    void* workspace, size_t ws_bytes, void* stream);
+DSA_API size_t dsa_index_prefill_pruned_paged_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                                              int n_seed);
+DSA_API int dsa_index_prefill_pruned_paged(const uint16_t* q, const float* w, const uint16_t* k_pages,
+                                           int64_t n_pages, int page_size, const int32_t* block_table,
+                                           int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                           const int32_t* seed_idx, int n_seed, int32_t* out_idx, float* out_score,
+                                           dsa_stats* stats, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Seed keys from historical selection frequency (163.com write-up, section
  * 03: a chunk's seed set may be the keys that earlier rows selected most).
  * Counts how often each key 0..n_keys-1 occurs in the Top-k lists of earlier

@@ -24,6 +24,8 @@ __all__ = [
     "dsa_index_prefill_pruned_workspace_bytes", "dsa_index_prefill_pruned_survivors",
     "dsa_index_prefill_host", "dsa_index_prefill_host_workspace_bytes", "dsa_test_inject_wait_timeout",
     "dsa_index_seeds_from_history", "dsa_index_seeds_from_history_workspace_bytes",
+    "dsa_index_prefill_paged", "dsa_index_prefill_paged_workspace_bytes",
+    "dsa_index_prefill_pruned_paged", "dsa_index_prefill_pruned_paged_workspace_bytes",
 ]
 
 DSA_OK = 0
@@ -76,6 +78,15 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
         L.dsa_index_prefill_pruned.restype = I
         L.dsa_index_prefill_pruned_survivors.argtypes = [P, I64, I64, I64, I, I, I, I, P, P, P, P]
         L.dsa_index_prefill_pruned_survivors.restype = I
+        L.dsa_index_prefill_paged_workspace_bytes.argtypes = [I64, I64, I, I, I]
+        L.dsa_index_prefill_paged_workspace_bytes.restype = SZ
+        L.dsa_index_prefill_paged.argtypes = [P, P, P, I64, I, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
+        L.dsa_index_prefill_paged.restype = I
+        L.dsa_index_prefill_pruned_paged_workspace_bytes.argtypes = [I64, I64, I, I, I, I]
+        L.dsa_index_prefill_pruned_paged_workspace_bytes.restype = SZ
+        L.dsa_index_prefill_pruned_paged.argtypes = [P, P, P, I64, I, P, I64, I64, I64, I, I, I, P, I, P, P, P, P,
+                                                     SZ, P]
+        L.dsa_index_prefill_pruned_paged.restype = I
         L.dsa_index_seeds_from_history_workspace_bytes.argtypes = [I64]
         L.dsa_index_seeds_from_history_workspace_bytes.restype = SZ
         L.dsa_index_seeds_from_history.argtypes = [P, I64, I, I64, I, P, P, SZ, P]
@@ -301,6 +312,77 @@ def dsa_index_prefill_pruned(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, 
                                               out_idx.data_ptr(), out_score.data_ptr(),
                                               ctypes.byref(st) if stats else None, ws.data_ptr(),
                                               ws.numel(), _stream_ptr(dev)))
+    if stats:
+        return out_idx, out_score, {f: int(getattr(st, f)) for f, _ in _Stats._fields_}
+    return out_idx, out_score
+
+
+def dsa_index_prefill_paged_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int) -> int:
+    return int(lib().dsa_index_prefill_paged_workspace_bytes(T_q, T_k, H, d, topk))
+
+
+def dsa_index_prefill_pruned_paged_workspace_bytes(T_q: int, T_k: int, H: int, d: int, topk: int,
+                                                   n_seed: int) -> int:
+    return int(lib().dsa_index_prefill_pruned_paged_workspace_bytes(T_q, T_k, H, d, topk, n_seed))
+
+
+def _paged_args(q, w, k_pages, block_table, dev):
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(w, "w", torch.float32, 2, dev)
+    _need(k_pages, "k_pages", torch.bfloat16, 3, dev)
+    _need(block_table, "block_table", torch.int32, 1, dev)
+    T_q, H, d = q.shape
+    n_pages, page_size, dk = k_pages.shape
+    if tuple(w.shape) != (T_q, H) or dk != d:
+        raise ValueError("shape mismatch between q (T_q,H,d), w (T_q,H) and k_pages (n_pages,page_size,d)")
+    return T_q, H, d, n_pages, page_size
+
+
+def dsa_index_prefill_paged(q: torch.Tensor, w: torch.Tensor, k_pages: torch.Tensor, block_table: torch.Tensor,
+                            q_offset: int, topk: int, T_k: int | None = None, out_idx=None, out_score=None,
+                            workspace=None):
+    """dsa_index_prefill over a paged key cache: key s of the sequence is
+    k_pages[block_table[s // page_size], s % page_size].  T_k defaults to
+    q_offset + T_q."""
+    dev = k_pages.device
+    T_q, H, d, n_pages, page_size = _paged_args(q, w, k_pages, block_table, dev)
+    T_k = int(q_offset) + T_q if T_k is None else int(T_k)
+    if block_table.shape[0] * page_size < T_k:
+        raise ValueError("block_table does not cover T_k keys")
+    out_idx, out_score = _outputs(T_q, topk, dev, out_idx, out_score)
+    ws = _workspace(dsa_index_prefill_paged_workspace_bytes(T_q, T_k, H, d, topk), dev, workspace)
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_paged(q.data_ptr(), w.data_ptr(), k_pages.data_ptr(), n_pages, page_size,
+                                             block_table.data_ptr(), int(q_offset), T_q, T_k, H, d, int(topk),
+                                             out_idx.data_ptr(), out_score.data_ptr(), ws.data_ptr(), ws.numel(),
+                                             _stream_ptr(dev)))
+    return out_idx, out_score
+
+
+def dsa_index_prefill_pruned_paged(q: torch.Tensor, w: torch.Tensor, k_pages: torch.Tensor,
+                                   block_table: torch.Tensor, q_offset: int, topk: int, seed_idx: torch.Tensor,
+                                   T_k: int | None = None, out_idx=None, out_score=None, workspace=None,
+                                   stats: bool = False):
+    """dsa_index_prefill_pruned over a paged key cache (see
+    dsa_index_prefill_paged for the page layout)."""
+    dev = k_pages.device
+    T_q, H, d, n_pages, page_size = _paged_args(q, w, k_pages, block_table, dev)
+    _need(seed_idx, "seed_idx", torch.int32, 1, dev)
+    T_k = int(q_offset) + T_q if T_k is None else int(T_k)
+    if block_table.shape[0] * page_size < T_k:
+        raise ValueError("block_table does not cover T_k keys")
+    n_seed = seed_idx.shape[0]
+    out_idx, out_score = _outputs(T_q, topk, dev, out_idx, out_score)
+    ws = _workspace(dsa_index_prefill_pruned_paged_workspace_bytes(T_q, T_k, H, d, topk, max(n_seed, 1)), dev,
+                    workspace)
+    st = _Stats()
+    with torch.cuda.device(dev):
+        _check(lib().dsa_index_prefill_pruned_paged(q.data_ptr(), w.data_ptr(), k_pages.data_ptr(), n_pages,
+                                                    page_size, block_table.data_ptr(), int(q_offset), T_q, T_k,
+                                                    H, d, int(topk), seed_idx.data_ptr(), n_seed,
+                                                    out_idx.data_ptr(), out_score.data_ptr(),
+                                                    ctypes.byref(st) if stats else None, ws.data_ptr(),
+                                                    ws.numel(), _stream_ptr(dev)))
     if stats:
         return out_idx, out_score, {f: int(getattr(st, f)) for f, _ in _Stats._fields_}
     return out_idx, out_score

@@ -567,6 +567,41 @@ int noalloc_scratch(void** out) {
   return DSA_OK;
 }
 
+// Paged prefill: the caller's workspace holds, in order, the workspace of
+// the contiguous call, the page gather's status word (256 bytes) and the
+// gathered keys [T_k][128] bf16.  The contiguous call's status word stays at
+// byte 0, where dsa_index_device_status reads it.
+size_t paged_tail_bytes(int64_t T_k) { return 256 + align_up(static_cast<size_t>(T_k) * kD * 2, 256); }
+
+int check_paged_pool(const uint16_t* k_pages, int64_t n_pages, int page_size, const int32_t* block_table) {
+  if (!k_pages || !block_table) return fail(DSA_EINVAL, "null pointer argument");
+  if (n_pages < 1 || page_size < 1) return fail(DSA_EINVAL, "need n_pages >= 1 and page_size >= 1");
+  if (n_pages * page_size >= (int64_t(1) << 31)) return fail(DSA_EINVAL, "n_pages * page_size must be below 2^31");
+  if (!aligned(k_pages, 16) || !aligned(block_table, 4))
+    return fail(DSA_EINVAL, "misaligned pointer (k_pages needs 16 bytes)");
+  return DSA_OK;
+}
+
+// Gathers the sequence's first T_k keys behind the contiguous workspace of
+// inner_bytes; returns the key matrix through *keys.
+int gather_paged_keys(const uint16_t* k_pages, int64_t n_pages, int page_size, const int32_t* block_table,
+                      int64_t T_k, uint8_t* ws, size_t inner_bytes, uint16_t** keys, cudaStream_t st) {
+  uint32_t* gst = reinterpret_cast<uint32_t*>(ws + inner_bytes);
+  *keys = reinterpret_cast<uint16_t*>(ws + inner_bytes + 256);
+  cudaError_t e = cudaMemsetAsync(gst, 0, 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  PageGatherParams gp{};
+  gp.k_pages = k_pages;
+  gp.n_pages = n_pages;
+  gp.page_size = page_size;
+  gp.block_table = block_table;
+  gp.T_k = T_k;
+  gp.k_out = *keys;
+  gp.status = gst;
+  if ((e = launch_page_gather(gp, sm_count(), st)) != cudaSuccess) return cuda_fail(e, "page gather launch");
+  return DSA_OK;
+}
+
 int check_prefill_args(int64_t q_offset, int64_t T_q, int64_t T_k, int H, int d, int topk) {
   int rc = check_shape(H, d, topk);
   if (rc != DSA_OK) return rc;
@@ -1182,6 +1217,77 @@ int dsa_index_prefill_pruned_survivors(const void* workspace, int64_t T_q, int64
       (e = cudaMemcpyAsync(row_state, ws + P.off_row_flags, static_cast<size_t>(T_q) * 4, cudaMemcpyDeviceToDevice,
                            st)) != cudaSuccess)
     return cuda_fail(e, "copying the screen's survivor mask");
+  return DSA_OK;
+}
+
+size_t dsa_index_prefill_paged_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk) {
+  const size_t inner = dsa_index_prefill_workspace_bytes(T_q, T_k, H, d, topk);
+  return inner ? align_up(inner, 256) + paged_tail_bytes(T_k) : 0;
+}
+
+int dsa_index_prefill_paged(const uint16_t* q, const float* w, const uint16_t* k_pages, int64_t n_pages,
+                            int page_size, const int32_t* block_table, int64_t q_offset, int64_t T_q, int64_t T_k,
+                            int H, int d, int topk, int32_t* out_idx, float* out_score, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  int rc = check_prefill_args(q_offset, T_q, T_k, H, d, topk);
+  if (rc != DSA_OK || T_q == 0) return rc;
+  if ((rc = check_paged_pool(k_pages, n_pages, page_size, block_table)) != DSA_OK) return rc;
+  if (!workspace || !aligned(workspace, 256)) return fail(DSA_EINVAL, "workspace must be 256-byte aligned");
+  const size_t tail = paged_tail_bytes(T_k);
+  if (ws_bytes < tail + 256) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed for the keys alone",
+                                         ws_bytes, tail + 256);
+  const size_t inner = (ws_bytes - tail) & ~static_cast<size_t>(255);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* keys = nullptr;
+  if ((rc = gather_paged_keys(k_pages, n_pages, page_size, block_table, T_k, ws, inner, &keys, st)) != DSA_OK)
+    return rc;
+  if ((rc = dsa_index_prefill(q, w, keys, q_offset, T_q, T_k, H, d, topk, out_idx, out_score, ws, inner, stream)) !=
+      DSA_OK)
+    return rc;
+  cudaError_t e = launch_status_or(reinterpret_cast<const uint32_t*>(ws + inner), reinterpret_cast<uint32_t*>(ws), st);
+  return e == cudaSuccess ? DSA_OK : cuda_fail(e, "status merge launch");
+}
+
+size_t dsa_index_prefill_pruned_paged_workspace_bytes(int64_t T_q, int64_t T_k, int H, int d, int topk,
+                                                      int n_seed) {
+  const size_t inner = dsa_index_prefill_pruned_workspace_bytes(T_q, T_k, H, d, topk, n_seed);
+  return inner ? align_up(inner, 256) + paged_tail_bytes(T_k) : 0;
+}
+
+int dsa_index_prefill_pruned_paged(const uint16_t* q, const float* w, const uint16_t* k_pages, int64_t n_pages,
+                                   int page_size, const int32_t* block_table, int64_t q_offset, int64_t T_q,
+                                   int64_t T_k, int H, int d, int topk, const int32_t* seed_idx, int n_seed,
+                                   int32_t* out_idx, float* out_score, dsa_stats* stats, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  int rc = check_prefill_args(q_offset, T_q, T_k, H, d, topk);
+  if (rc != DSA_OK) return rc;
+  if ((rc = check_paged_pool(k_pages, n_pages, page_size, block_table)) != DSA_OK) return rc;
+  if (!workspace || !aligned(workspace, 256)) return fail(DSA_EINVAL, "workspace must be 256-byte aligned");
+  const size_t tail = paged_tail_bytes(T_k);
+  const size_t need = dsa_index_prefill_pruned_paged_workspace_bytes(T_q, T_k, H, d, topk, n_seed);
+  if (need == 0) return fail(DSA_EINVAL, "bad sizes");
+  if (ws_bytes < need) return fail(DSA_EWORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  const size_t inner = need - tail;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* keys = nullptr;
+  if (T_q > 0 &&
+      (rc = gather_paged_keys(k_pages, n_pages, page_size, block_table, T_k, ws, inner, &keys, st)) != DSA_OK)
+    return rc;
+  if ((rc = dsa_index_prefill_pruned(q, w, keys ? keys : k_pages, q_offset, T_q, T_k, H, d, topk, seed_idx, n_seed,
+                                     out_idx, out_score, stats, ws, inner, stream)) != DSA_OK)
+    return rc;
+  if (T_q == 0) return DSA_OK;
+  cudaError_t e = launch_status_or(reinterpret_cast<const uint32_t*>(ws + inner), reinterpret_cast<uint32_t*>(ws), st);
+  if (e != cudaSuccess) return cuda_fail(e, "status merge launch");
+  if (stats) {  // the pruned call synchronised before the merge: read the gather's bit as well
+    uint32_t s = 0;
+    if ((e = cudaMemcpyAsync(&s, ws + inner, 4, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      return cuda_fail(e, "reading the page gather status");
+    if (s) return fail(DSA_EDEVICE, "a block-table entry lies outside the page pool (status 0x%x)", s);
+  }
   return DSA_OK;
 }
 

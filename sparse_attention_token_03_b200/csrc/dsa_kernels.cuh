@@ -262,6 +262,19 @@ cudaError_t launch_refine_shared(int H, const CUtensorMap& tmap_q, const CUtenso
 cudaError_t launch_screen(const CUtensorMap& tmap_plan, const CUtensorMap& tmap_k, const ScoreParams& p,
                           int grid, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+
+// Paged key cache -> contiguous keys (dsa_pages.cu).
+struct PageGatherParams {
+  const uint16_t* k_pages;      // [n_pages][page_size][128]
+  int64_t n_pages;
+  int page_size;
+  const int32_t* block_table;   // [ceil(T_k / page_size)] page ids of the sequence
+  int64_t T_k;
+  uint16_t* k_out;              // [T_k][128]
+  uint32_t* status;             // status word (overflow bit on a bad page id)
+};
+cudaError_t launch_page_gather(const PageGatherParams& p, int sms, cudaStream_t st);
+cudaError_t launch_status_or(const uint32_t* src, uint32_t* dst, cudaStream_t st);
 cudaError_t launch_decode_plan(const DecodePlanParams& p, cudaStream_t stream);
 
 }  // namespace dsa

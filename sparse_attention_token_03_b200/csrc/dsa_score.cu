@@ -93,6 +93,46 @@ __device__ void epi_find_bucket(const uint32_t* hist, int nb, int above, int nee
   epi_sync(bar);
 }
 
+// Threshold update with two barriers: the thread holding the topk-th record's
+// bin raises the threshold itself.
+__device__ void epi_raise(const uint32_t* hist, int need, int tid, int* scratch, int* res, uint64_t* thr,
+                          int* upd, int total, int bar) {
+  constexpr int bpt = kHistBins / kEpiThreads;
+  const int lo = tid * bpt;
+  int local = 0;
+#pragma unroll
+  for (int b = 0; b < bpt; ++b) local += hist[lo + b];
+  const int lane = tid & 31, wid = tid >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += v;
+  }
+  if (lane == 0) scratch[wid] = incl;
+  epi_sync(bar);
+  int higher_warps = 0;
+  for (int w2 = wid + 1; w2 < kEpiThreads / 32; ++w2) higher_warps += scratch[w2];
+  const int excl = incl - local + higher_warps;
+  if (excl < need && excl + local >= need) {
+    int acc = excl;
+    for (int b = bpt - 1; b >= 0; --b) {
+      const int h = hist[lo + b];
+      if (acc + h >= need) {
+        res[0] = lo + b;
+        res[1] = acc;
+        res[2] = h;
+        const uint64_t t_new = static_cast<uint64_t>(hist_edge(static_cast<uint32_t>(lo + b))) << 32;
+        if (t_new > *thr) *thr = t_new;
+        *upd = total;
+        break;
+      }
+      acc += h;
+    }
+  }
+  epi_sync(bar);
+}
+
 // Exact fallback compaction of one (slot, query), run by its epilogue
 // warpgroup when the histogram threshold would keep too many records.  The records of the active half (base region + four append
 // regions) are reduced to a superset of the `need` largest ones holding at
@@ -830,15 +870,8 @@ __global__ void __launch_bounds__(score_threads(EG), 1)
           // bin B is beaten by topk records and can never be selected.
           int kept_above = 0;
           if (total >= p.topk && (full || total - s_upd[qq] >= 256)) {
-            epi_find_bucket(qh, kHistBins, 0, p.topk, etid, s_misc + 4, s_misc + 1, bar);
-            const uint64_t t_new = static_cast<uint64_t>(hist_edge(static_cast<uint32_t>(s_misc[1]))) << 32;
+            epi_raise(qh, p.topk, etid, s_misc + 4, s_misc + 1, &s_thr[qq], &s_upd[qq], total, bar);
             kept_above = s_misc[2] + s_misc[3];
-            epi_sync(bar);
-            if (etid == 0) {
-              if (t_new > s_thr[qq]) s_thr[qq] = t_new;
-              s_upd[qq] = total;
-            }
-            epi_sync(bar);
           }
           if (!full) continue;
           const int half_q = s_half[qq];

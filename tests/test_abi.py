@@ -113,3 +113,21 @@ def test_history_seeds_validation_without_gpu():
     assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 5, dummy, P(264), need, None) == -1
     small = L.dsa_index_seeds_from_history_workspace_bytes(10)
     assert L.dsa_index_seeds_from_history(dummy, 4, 8, 10, 5, dummy, dummy, small - 1, None) == -3
+
+
+def test_paged_prefill_validation_without_gpu():
+    L = dsa.lib()
+    P = ctypes.c_void_p
+    d = P(256)
+    need = L.dsa_index_prefill_paged_workspace_bytes(256, 1024, 64, 128, 64)
+    # the contiguous call's workspace plus the status block and 1024 gathered keys
+    assert need >= L.dsa_index_prefill_workspace_bytes(256, 1024, 64, 128, 64) + 256 + 1024 * 256
+    assert L.dsa_index_prefill_pruned_paged_workspace_bytes(256, 1024, 64, 128, 64, 128) >= \
+        L.dsa_index_prefill_pruned_workspace_bytes(256, 1024, 64, 128, 64, 128) + 1024 * 256
+    # unsupported heads, bad page sizes, null pools and misaligned workspaces fail before any CUDA call
+    assert L.dsa_index_prefill_paged(d, d, d, 8, 128, d, 768, 256, 1024, 48, 128, 64, d, d, d, need, None) == -2
+    assert L.dsa_index_prefill_paged(d, d, d, 8, 0, d, 768, 256, 1024, 64, 128, 64, d, d, d, need, None) == -1
+    assert L.dsa_index_prefill_paged(d, d, None, 8, 128, d, 768, 256, 1024, 64, 128, 64, d, d, d, need, None) == -1
+    assert L.dsa_index_prefill_paged(d, d, d, 8, 128, d, 768, 256, 1024, 64, 128, 64, d, d, P(264), need,
+                                     None) == -1
+    assert L.dsa_index_prefill_paged(d, d, d, 8, 128, d, 768, 256, 1024, 64, 128, 64, d, d, d, 1000, None) == -3

@@ -77,3 +77,76 @@ def test_paged_decode_long_caches_match_contiguous():
     pi, ps = dsa.dsa_index_decode_paged(q, w, _bf16(pool), torch.from_numpy(bt).cuda(), sl, 2048)
     torch.cuda.synchronize()
     assert torch.equal(pi, ci) and torch.equal(ps.view(torch.int32), cs.view(torch.int32))
+
+
+def sequence_pages(k, page, seed, spare_pages=2):
+    """One sequence's keys (T_k, d) scattered over a shuffled page pool;
+    returns the pool (n_pages, page, d) and the block table (n_blocks,)."""
+    T_k, d = k.shape
+    n_blocks = (T_k + page - 1) // page
+    n_pages = n_blocks + spare_pages
+    rng = np.random.default_rng(seed)
+    bt = rng.permutation(n_pages)[:n_blocks].astype(np.int32)
+    pool = rng.integers(0, 2 ** 15, size=(n_pages, page, d)).astype(np.uint16)  # unused pages: junk
+    padded = np.zeros((n_blocks * page, d), np.uint16)
+    padded[:T_k] = k
+    pool[bt] = padded.reshape(n_blocks, page, d)
+    return pool, bt
+
+
+@pytest.mark.parametrize("page,T_q,T_k", [(64, 700, 2500), (16, 300, 1000), (1000, 512, 3000)])
+def test_paged_prefill_equals_contiguous(page, T_q, T_k):
+    from synth import make_prefill
+    x = make_prefill("causal_16k_h64", T_q=T_q, T_k=T_k, q_offset=T_k - T_q, seed=71)
+    pool, bt = sequence_pages(x["k"], page, seed=72)
+    q, w = _bf16(x["q"]), torch.from_numpy(x["w"]).cuda()
+    for topk in (2048, 77):
+        ci, cs = dsa.dsa_index_prefill(q, w, _bf16(x["k"]), T_k - T_q, topk)
+        pi, ps = dsa.dsa_index_prefill_paged(q, w, _bf16(pool), torch.from_numpy(bt).cuda(), T_k - T_q, topk)
+        torch.cuda.synchronize()
+        assert torch.equal(pi, ci) and torch.equal(ps.view(torch.int32), cs.view(torch.int32))
+
+
+def test_paged_prefill_row_blocks_in_a_small_workspace():
+    # a workspace below the full size: the keys are gathered once and the
+    # rows run in blocks; the result is unchanged
+    from synth import make_prefill
+    T_q = T_k = 4096
+    x = make_prefill("causal_16k_h64", T_q=T_q, T_k=T_k, q_offset=0, seed=73)
+    pool, bt = sequence_pages(x["k"], 128, seed=74)
+    q, w = _bf16(x["q"]), torch.from_numpy(x["w"]).cuda()
+    full = dsa.dsa_index_prefill_paged_workspace_bytes(T_q, T_k, 64, 128, 2048)
+    ws = torch.empty(full // 3, dtype=torch.uint8, device="cuda")
+    ci, cs = dsa.dsa_index_prefill(q, w, _bf16(x["k"]), 0, 2048)
+    pi, ps = dsa.dsa_index_prefill_paged(q, w, _bf16(pool), torch.from_numpy(bt).cuda(), 0, 2048, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(pi, ci) and torch.equal(ps.view(torch.int32), cs.view(torch.int32))
+
+
+def test_paged_pruned_equals_contiguous_pruned():
+    from synth import make_prefill, random_distinct_keys
+    T_k, T_q, topk = 6000, 512, 512
+    x = make_prefill("chunk_128k_h32", T_q=T_q, T_k=T_k, q_offset=T_k - T_q, seed=75)
+    pool, bt = sequence_pages(x["k"], 64, seed=76)
+    seeds = torch.from_numpy(random_distinct_keys(77, 0, T_k - T_q, 1536)).cuda()
+    q, w = _bf16(x["q"]), torch.from_numpy(x["w"]).cuda()
+    ci, cs, cst = dsa.dsa_index_prefill_pruned(q, w, _bf16(x["k"]), T_k - T_q, topk, seeds, stats=True)
+    pi, ps, pst = dsa.dsa_index_prefill_pruned_paged(q, w, _bf16(pool), torch.from_numpy(bt).cuda(), T_k - T_q,
+                                                     topk, seeds, stats=True)
+    di, ds = dsa.dsa_index_prefill(q, w, _bf16(x["k"]), T_k - T_q, topk)
+    torch.cuda.synchronize()
+    assert torch.equal(pi, ci) and torch.equal(ps.view(torch.int32), cs.view(torch.int32))
+    assert torch.equal(pi, di) and torch.equal(ps.view(torch.int32), ds.view(torch.int32))
+    assert pst == cst
+
+
+def test_paged_prefill_flags_a_bad_page_id():
+    from synth import make_prefill
+    x = make_prefill("causal_16k_h64", T_q=256, T_k=1024, q_offset=768, seed=78)
+    pool, bt = sequence_pages(x["k"], 64, seed=79)
+    bt[3] = pool.shape[0] + 7  # outside the pool
+    q, w = _bf16(x["q"]), torch.from_numpy(x["w"]).cuda()
+    ws = torch.empty(dsa.dsa_index_prefill_paged_workspace_bytes(256, 1024, 64, 128, 64), dtype=torch.uint8,
+                     device="cuda")
+    dsa.dsa_index_prefill_paged(q, w, _bf16(pool), torch.from_numpy(bt).cuda(), 768, 64, workspace=ws)
+    assert dsa.dsa_index_device_status(ws) & 2
