@@ -347,9 +347,51 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
     }
   }
   __syncthreads();
-  const int n = s_n;  // records at or above the row threshold
+  int n = s_n;  // records at or above the row threshold
   const int m = min(p.topk, n);
-  const bool staged = n <= kSelStage;
+  bool staged = n <= kSelStage;
+
+  // 2b. more records than the staging buffer holds: count all of them over
+  //     the linear score digit of the counting path (range [s_lo, s_hi]),
+  //     find the bucket B of the m-th, and stage again only the records in
+  //     buckets >= B (every one of the m winners, usually a few more); the
+  //     counting path then runs on them unchanged
+  if (!staged && m > 0 && table) {
+    const float smin = record_score(s_lo), srange = record_score(s_hi) - smin;
+    const float scale = static_cast<float>(kSelBins - 1) / srange;
+    if (srange >= 1e-30f && srange <= 3.0e38f && scale <= 3.0e38f) {
+      auto digit = [&](uint64_t r) {
+        return min(static_cast<uint32_t>(kSelBins - 1), static_cast<uint32_t>((record_score(r) - smin) * scale));
+      };
+      for (int i = tid; i < kSelBins; i += NT) s_hist[i] = 0u;
+      __syncthreads();
+      // one pass over the row's records: f(valid, record) for index tid, tid + NT, ...
+      auto for_records = [&](auto&& f) {
+        int sg = 0;
+        for (int base = 0; base < total; base += NT) {
+          const int i = base + tid;
+          uint64_t r = 0ull;
+          if (i < total) {
+            while (s_segoff[sg + 1] <= i) ++sg;
+            r = s_segptr[sg][i - s_segoff[sg]];
+          }
+          f(i < total && r != 0ull && r >= thr, r);
+        }
+      };
+      for_records([&](bool in, uint64_t r) {
+        if (in) atomicAdd(&s_hist[digit(r)], 1u);
+      });
+      __syncthreads();
+      find_bucket_blk<NT>(s_hist, kSelBins, 0, m, s_scratch, s_res);
+      const uint32_t B = static_cast<uint32_t>(s_res[0]);
+      if (tid == 0) s_n = 0;
+      __syncthreads();
+      for_records([&](bool in, uint64_t r) { stage_append(in && digit(r) >= B, r, s_rec, kSelStage, &s_n, lane); });
+      __syncthreads();
+      n = s_n;
+      staged = n <= kSelStage;
+    }
+  }
 
   const size_t o = static_cast<size_t>(row) * p.topk;
   const size_t orec = static_cast<size_t>(row) * p.rec_stride;
