@@ -513,40 +513,24 @@ __global__ void __launch_bounds__(NT, 4) select_topk_kernel(const SelectParams p
         if (static_cast<int>(d) >= B) s_rec[atomicAdd(&s_cur[d], 1u)] = v[j];
       }
       __syncthreads();
-      // s_cur[d] is now the end of bucket d; rank each winner inside its
-      // bucket and place it at its final position of the output
-      for (int base = tid; base < nw; base += kBatch * NT) {
-        uint64_t r[kBatch];
-        int beg[kBatch], end[kBatch];
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) r[j] = base + j * NT < nw ? s_rec[base + j * NT] : 0ull;
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-          const uint32_t d = r[j] != 0ull ? digit(r[j]) : 0u;
-          end[j] = static_cast<int>(s_cur[d]);
-          beg[j] = r[j] != 0ull ? end[j] - static_cast<int>(s_hist[d]) : end[j];
+      // s_cur[d] is now the end of bucket d; each thread ranks one winner at
+      // a time inside its own bucket (consecutive threads hold consecutive
+      // winners, so a warp scans about one bucket's length) and writes it
+      // straight to its final position of the output
+      for (int i = tid; i < nw; i += NT) {
+        const uint64_t r = s_rec[i];
+        const uint32_t d = digit(r);
+        const int end = static_cast<int>(s_cur[d]);
+        const int beg = end - static_cast<int>(s_hist[d]);
+        int rank = 0;
+        for (int x = beg; x < end; x += 2) {
+          const uint64_t a0 = s_rec[x];
+          const uint64_t a1 = x + 1 < end ? s_rec[x + 1] : 0ull;
+          rank += (a0 > r ? 1 : 0) + (a1 > r ? 1 : 0);
         }
-        // the batch's bucket scans advance together (independent loads)
-        int rank[kBatch], len = 0;
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-          rank[j] = 0;
-          len = max(len, end[j] - beg[j]);
-        }
-        for (int x = 0; x < len; x += 2) {
-#pragma unroll
-          for (int j = 0; j < kBatch; ++j) {
-            const uint64_t a0 = beg[j] + x < end[j] ? s_rec[beg[j] + x] : 0ull;
-            const uint64_t a1 = beg[j] + x + 1 < end[j] ? s_rec[beg[j] + x + 1] : 0ull;
-            rank[j] += (a0 > r[j] ? 1 : 0) + (a1 > r[j] ? 1 : 0);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j)
-          if (r[j] != 0ull && beg[j] + rank[j] < m) s_out[beg[j] + rank[j]] = r[j];
+        if (beg + rank < m) put(beg + rank, r);
       }
-      __syncthreads();
-      for (int i = tid; i < p.topk; i += NT) put(i, i < m ? s_out[i] : 0ull);
+      for (int i = m + tid; i < p.topk; i += NT) put(i, 0ull);
       done = true;
     }
     __syncthreads();
