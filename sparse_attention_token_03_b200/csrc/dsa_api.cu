@@ -195,9 +195,10 @@ PrefillPlan plan_prefill(int64_t T_q, int64_t T_k, int64_t q_offset_hint, int H,
   }
   P.n_units = P.n_groups * P.S;
   // Epilogue width: four warpgroups (one query each at H = 64) hide the
-  // admission work of units whose keys are few per selected record; with
-  // many keys per record admissions are rare, the head sums dominate and two
-  // warpgroups with the head weights in registers issue fewer instructions.
+  // admission work and keep 16 weights per thread in registers; only for
+  // units of very many keys per selected record, where admissions are rare
+  // and the head sums dominate, two warpgroups with all head weights in
+  // registers are used.
   const double unit_keys = (static_cast<double>(std::max<int64_t>(q_offset_hint, 0)) +
                             0.5 * static_cast<double>(T_q + 1)) / P.S;
   P.eg = unit_keys >= static_cast<double>(kWideKeysPerRecord) * topk ? 2 : 4;

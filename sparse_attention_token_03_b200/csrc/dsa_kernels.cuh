@@ -39,8 +39,9 @@ static_assert(128 * regs_ctl(4) + 512 * regs_epi(4) <= 640 * regs_launch(4), "re
 static_assert(regs_launch(2) * 384 <= 65536 && regs_launch(4) * 640 <= 65536, "launch registers");
 constexpr int kSelectThreads = 256;
 // A grouped prefill unit whose keys number at least this many times topk
-// runs the two-warpgroup epilogue, shorter ones the four-warpgroup one.
-constexpr int kWideKeysPerRecord = 256;
+// runs the two-warpgroup epilogue, shorter ones the four-warpgroup one
+// (measured: four warpgroups are faster up to 1M keys at topk = 2048).
+constexpr int kWideKeysPerRecord = 2048;
 
 constexpr int kMetaInts = 8;
 // Score-code histogram of a query's buffered records, 1024 bins: 1/8-octave
