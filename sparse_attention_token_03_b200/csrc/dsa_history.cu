@@ -5,7 +5,7 @@
 // Given the Top-k index lists of earlier rows, the seeds are the n_seed keys
 // below n_keys with the largest selection counts, ties going to the smaller
 // key, written in ascending key order.  An exact top-n_seed by
-// (count desc, key asc) over a count array, in five steps:
+// (count desc, key asc) over a count array:
 //
 //   count_kernel      counts[s] += 1 for every list entry s in [0, n_keys)
 //   hist_kernel x2    radix histogram of the counts, high then low 16 bits
